@@ -1,0 +1,217 @@
+"""Seeded synthetic q, k, v for the TriangleMix workloads.
+
+This module draws numbers and nothing else: no masking, no softmax, no
+attention arithmetic. Both the CUDA path and the CPU oracle are fed from it,
+so they always see the same bf16 bytes.
+
+The pages measure on model activations of Llama-3-8B / Qwen2.5-7B running
+LongBench, RULER and Wikipedia text (TriangleMix blog post, sections 性能 and
+缘由; 36kr interview, "Darstellung der Messergebnisse"). None of those are
+available here; seeded tensors with the models' attention shapes stand in for
+them. The value recipe per workload:
+
+* plain:    q, k, v ~ N(0, 1) rounded to bf16.
+* outliers: as plain, then for every kv head g four distinct channels are
+            multiplied by 8 in k[..., g, :] and in every q head of g's group
+            (the same channels in q and k, so they raise the logits).
+* headscale: q and k heads each get their own factor ~ U[0.5, 2].
+
+Element values come from the C generator in ``tm_inputs.c`` (splitmix64 +
+Box-Muller, bf16 round-to-nearest-even). Channel choices and head factors are
+drawn here from the same splitmix64 finaliser so that they are identical on
+every machine.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass, field
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libtm_inputs.so")
+_lib = None
+
+TENSOR_Q, TENSOR_K, TENSOR_V = 0, 1, 2
+_M64 = (1 << 64) - 1
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                f"{_LIB_PATH} is missing: run `python -c 'import __graft_entry__ as g; g.build()'`")
+        lib = ctypes.CDLL(_LIB_PATH)
+        lib.tm_inputs_fill_bf16.restype = ctypes.c_int
+        lib.tm_inputs_fill_bf16.argtypes = [
+            ctypes.c_void_p, ctypes.c_longlong, ctypes.c_longlong, ctypes.c_int, ctypes.c_int,
+            ctypes.c_uint64, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+        lib.tm_inputs_normal_at.restype = ctypes.c_double
+        lib.tm_inputs_normal_at.argtypes = [ctypes.c_uint64, ctypes.c_uint64]
+        lib.tm_inputs_stream_key.restype = ctypes.c_uint64
+        lib.tm_inputs_stream_key.argtypes = [ctypes.c_uint64, ctypes.c_int]
+        _lib = lib
+    return _lib
+
+
+def _mix64(z: int) -> int:
+    z = (z + 0x9E3779B97F4A7C15) & _M64
+    z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & _M64
+    z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & _M64
+    return z ^ (z >> 31)
+
+
+def _uniform(seed: int, stream: int, n: int) -> float:
+    """Uniform in [0, 1) from the splitmix64 stream (seed, stream), draw n."""
+    key = _mix64(_mix64(seed) ^ _mix64(stream + 0x5151))
+    return (_mix64((key + n) & _M64) >> 11) * (1.0 / (1 << 53))
+
+
+def default_threads() -> int:
+    return max(1, min(64, os.cpu_count() or 1))
+
+
+def fill_bf16(out, B: int, N: int, H: int, D: int, seed: int, tensor_id: int,
+              head_scale=None, chan_scale=None, nthreads: int | None = None):
+    """Fill ``out`` (numpy uint16 array or raw host pointer int) for a [B, N, H, D] tensor."""
+    lib = _load()
+    if isinstance(out, np.ndarray):
+        assert out.dtype == np.uint16 and out.flags.c_contiguous and out.size == B * N * H * D
+        ptr = out.ctypes.data
+    else:
+        ptr = int(out)
+    hs = None if head_scale is None else np.ascontiguousarray(head_scale, dtype=np.float32)
+    cs = None if chan_scale is None else np.ascontiguousarray(chan_scale, dtype=np.float32)
+    rc = lib.tm_inputs_fill_bf16(
+        ctypes.c_void_p(ptr), B, N, H, D, ctypes.c_uint64(seed & _M64), tensor_id,
+        None if hs is None else ctypes.c_void_p(hs.ctypes.data),
+        None if cs is None else ctypes.c_void_p(cs.ctypes.data),
+        nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("tm_inputs_fill_bf16: bad argument")
+    return out
+
+
+def normal_at(seed: int, tensor_id: int, n: int) -> float:
+    """The unrounded normal sample behind flat element n (for generator self-tests)."""
+    lib = _load()
+    return lib.tm_inputs_normal_at(lib.tm_inputs_stream_key(seed & _M64, tensor_id), n)
+
+
+@dataclass(frozen=True)
+class Workload:
+    """One attention workload: shapes, triangle parameters and value recipe."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    N: int
+    D: int
+    S: int
+    W: int
+    L: int
+    layers: int = 1
+    tri_start: int = 0
+    recipe: str = "plain"          # plain | outliers | headscale
+    seed_is_layer: bool = False
+    windows: tuple = field(default=())
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / float(np.sqrt(self.D))
+
+    def seed(self, layer: int) -> int:
+        return layer if self.seed_is_layer else 0
+
+
+# The five workloads: shapes of Llama-3-8B (32 q heads, 8 kv heads, head dim
+# 128, 32 layers) and Qwen2.5-7B (28 q heads, 4 kv heads, 28 layers) with the
+# layer splits the blog post reports (12 dense layers for Llama-3, 20 for
+# Qwen2.5; section 性能) and triangle parameters S/W/L chosen per workload.
+WORKLOADS = {
+    "tiny": Workload("tiny", B=1, Hq=4, Hkv=4, N=512, D=64, S=16, W=64, L=64,
+                     layers=2, tri_start=1),
+    "llama3-8b-32k": Workload("llama3-8b-32k", B=1, Hq=32, Hkv=8, N=32768, D=128,
+                              S=64, W=1024, L=128, layers=2, tri_start=1, recipe="outliers"),
+    "llama3-8b-64k-32layer": Workload("llama3-8b-64k-32layer", B=1, Hq=32, Hkv=8, N=65536,
+                                      D=128, S=64, W=1024, L=128, layers=32, tri_start=12,
+                                      seed_is_layer=True),
+    "llama3-8b-128k": Workload("llama3-8b-128k", B=1, Hq=32, Hkv=8, N=131072, D=128,
+                               S=64, W=2048, L=256, layers=2, tri_start=1,
+                               windows=(512, 1024, 2048, 4096)),
+    "qwen2.5-7b-128k-28layer": Workload("qwen2.5-7b-128k-28layer", B=1, Hq=28, Hkv=4,
+                                        N=131072, D=128, S=64, W=1024, L=128, layers=28,
+                                        tri_start=20, recipe="headscale"),
+}
+
+
+def outlier_channels(seed: int, Hkv: int, D: int, count: int = 4):
+    """Per kv head, ``count`` distinct channels drawn without replacement."""
+    chans = []
+    for g in range(Hkv):
+        picked, n = [], 0
+        while len(picked) < count:
+            c = int(_uniform(seed, 1000 + g, n) * D)
+            n += 1
+            if c not in picked:
+                picked.append(c)
+        chans.append(sorted(picked))
+    return chans
+
+
+def head_scales(seed: int, H: int, stream: int):
+    return np.array([0.5 + 1.5 * _uniform(seed, stream, h) for h in range(H)], dtype=np.float32)
+
+
+def scales_for(wl: Workload, layer: int = 0):
+    """(head_scale, chan_scale) for q, k, v under the workload's recipe."""
+    seed = wl.seed(layer)
+    none = (None, None)
+    if wl.recipe == "plain":
+        return none, none, none
+    if wl.recipe == "outliers":
+        G = wl.Hq // wl.Hkv
+        cq = np.ones((wl.Hq, wl.D), np.float32)
+        ck = np.ones((wl.Hkv, wl.D), np.float32)
+        for g, chans in enumerate(outlier_channels(seed, wl.Hkv, wl.D)):
+            for c in chans:
+                ck[g, c] = 8.0
+                cq[g * G:(g + 1) * G, c] = 8.0
+        return (None, cq.reshape(-1)), (None, ck.reshape(-1)), none
+    if wl.recipe == "headscale":
+        return (head_scales(seed, wl.Hq, 2000), None), (head_scales(seed, wl.Hkv, 2001), None), none
+    raise ValueError(wl.recipe)
+
+
+def make_qkv(wl: Workload, layer: int = 0, out=None, N: int | None = None, nthreads=None):
+    """Return (q, k, v) as uint16 arrays of bf16 bits, shapes [B,N,Hq,D], [B,N,Hkv,D] x2.
+
+    ``out`` may be a tuple of three preallocated uint16 arrays (e.g. views of
+    pinned host tensors). ``N`` overrides the workload's sequence length.
+    """
+    N = wl.N if N is None else N
+    seed = wl.seed(layer)
+    (qh, qc), (kh, kc), (vh, vc) = scales_for(wl, layer)
+    shapes = [(wl.B, N, wl.Hq, wl.D), (wl.B, N, wl.Hkv, wl.D), (wl.B, N, wl.Hkv, wl.D)]
+    if out is None:
+        out = tuple(np.empty(s, np.uint16) for s in shapes)
+    for arr, shp, tid, hs, cs in zip(out, shapes, (TENSOR_Q, TENSOR_K, TENSOR_V),
+                                    (qh, kh, vh), (qc, kc, vc)):
+        fill_bf16(arr.reshape(-1), *shp[:2], shp[2], shp[3], seed, tid, hs, cs, nthreads)
+    return out
+
+
+def bf16_bits_to_f32(a: np.ndarray) -> np.ndarray:
+    return (a.astype(np.uint32) << 16).view(np.float32)
+
+
+def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """Round-to-nearest-even float32 -> bf16 bits (NaN kept quiet)."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    nan = (u & 0x7F800000) == 0x7F800000
+    nan &= (u & 0x007FFFFF) != 0
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+    r[nan] = ((u[nan] >> 16) | 0x40).astype(np.uint16)
+    return r
