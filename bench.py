@@ -1,0 +1,335 @@
+#!/usr/bin/env python
+"""Benchmark of TriangleMix prefill attention on B200.
+
+One step = one pass of the TriangleMix layer schedule over one batch of
+synthetic inputs of the named workload: the triangle layer (layer index =
+tri_start) and the dense causal layer just below it (tri_start - 1), both
+through ``tm_trianglemix_attn_fwd``. The headline metric is the triangle
+kernel's throughput counting only the FLOPs of the tiles it visits (4*BM*BN*D
+per kept 128x128 tile per q head); the causal kernel's time gives the speedup.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+With N > 1 (under torchrun) every rank runs an independent replica: the path
+shards by (batch, kv-head group) with no exchange, so there is no data-path
+collective; only the timing is reduced (max over ranks).
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_prefill_trianglemix_b200 import inputs as I  # noqa: E402
+
+METRIC = "triangle-attn prefill TFLOP/s (kept tiles) at 128K; speedup vs own causal"
+UNIT = "TFLOP/s"
+BM = BN = 128
+# Per-launch DRAM traffic of the triangle kernel from an ncu capture, keyed by
+# the hash of the kernel sources it was taken on (reported only while they match).
+TRAFFIC = {}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "long_context_prefill_trianglemix_b200", "csrc",
+                                           "*"))):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"burst": float(d["bf16_tflops"]), "sustained": float(d["bf16_tflops_sustained"]),
+                "hbm": float(d["hbm_gbs"]), "source": "measured"}
+    except Exception:
+        return {"burst": 1590.0, "sustained": 1400.0, "hbm": 6650.0, "source": "fallback"}
+
+
+def tile_flop(wl, causal, W=None) -> float:
+    import long_context_prefill_trianglemix_b200 as tm
+    tiles = tm.tm_kept_tiles(wl.N, causal, wl.S, wl.W if W is None else W, wl.L)
+    return float(tiles) * wl.B * wl.Hq * 4.0 * BM * BN * wl.D
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="tm_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        busy = [s for s in sm if s > 0.5 * (max(mx) if mx else 1)]
+        return {"sm_mhz": statistics.median(busy or sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def oracle_sample(wl, W, n_rows: int, seed: int, host):
+    """Time the fp64 oracle on a row sample of the triangle layer; returns
+    (seconds, tile-FLOP equivalent of the sample, cores, description)."""
+    import numpy as np
+
+    import oracle
+    import long_context_prefill_trianglemix_b200 as tm
+    q, k, v = host
+    rng = np.random.default_rng(seed)
+    rows = sorted(rng.choice(wl.N, size=n_rows, replace=False).tolist())
+    tiles = tm.tm_tile_list(wl.N, False, wl.S, W, wl.L)
+    per_qb = np.bincount(tiles[:, 0], minlength=(wl.N + BM - 1) // BM)
+    cores = oracle.hardware_threads()
+    t0 = time.perf_counter()
+    oracle.attention(q, k, v, wl.B, wl.Hq, wl.Hkv, wl.N, wl.D, wl.scale, False, wl.S, W, wl.L,
+                     rows=rows, nthreads=cores)
+    dt = time.perf_counter() - t0
+    # each sampled row stands for its share (1/BM) of its q-block's kept tiles
+    equiv = float(sum(per_qb[r // BM] for r in rows)) * BN * 4.0 * wl.D * wl.Hq * wl.B
+    desc = (f"{n_rows} seeded random query rows x all {wl.Hq} q heads of the triangle layer "
+            f"(W={W}); credited with their share of the kept-tile FLOPs")
+    return dt, equiv, cores, desc
+
+
+# ----------------------------------------------------------------------------- arms
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def run_reference(args):
+    ws, rank, _ = dist_setup()
+    if rank != 0:
+        return 0
+    wl = I.WORKLOADS[args.workload]
+    W = args.window or wl.W
+    host = I.make_qkv(wl)
+    for s in range(args.warmup):
+        oracle_sample(wl, W, args.ref_rows, 1000 + s, host)
+    tot_t, tot_f = 0.0, 0.0
+    desc, cores = "", 1
+    for s in range(args.steps):
+        dt, equiv, cores, desc = oracle_sample(wl, W, args.ref_rows, s, host)
+        tot_t += dt
+        tot_f += equiv
+    value = tot_f / tot_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "N": wl.N,
+                   "D": wl.D, "S": wl.S, "W": W, "L": wl.L},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import long_context_prefill_trianglemix_b200 as tm
+
+    ws, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    if ws > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    wl = I.WORKLOADS[args.workload]
+    W = args.window or wl.W
+    tri_layer, causal_layer = wl.tri_start, max(wl.tri_start - 1, 0)
+    assert wl.tri_start >= 1
+
+    # pinned host inputs (filled in place by the seeded generator), then device copies
+    shp_q, shp_kv = (wl.B, wl.N, wl.Hq, wl.D), (wl.B, wl.N, wl.Hkv, wl.D)
+    hq = torch.empty(shp_q, dtype=torch.int16, pin_memory=True)
+    hk = torch.empty(shp_kv, dtype=torch.int16, pin_memory=True)
+    hv = torch.empty(shp_kv, dtype=torch.int16, pin_memory=True)
+    host_np = tuple(t.numpy().view(np.uint16) for t in (hq, hk, hv))
+    I.make_qkv(wl, tri_layer, out=host_np)
+    dq, dk, dv = (t.cuda().view(torch.bfloat16) for t in (hq, hk, hv))
+    do = torch.empty_like(dq)
+    ho = torch.empty(shp_q, dtype=torch.int16, pin_memory=True)
+    stream = torch.cuda.current_stream()
+
+    def layer_call(layer, q=dq, k=dk, v=dv, o=do):
+        tm.tm_trianglemix_attn_fwd(q, k, v, o, wl.B, wl.Hq, wl.Hkv, wl.N, wl.D, wl.scale,
+                                   wl.S, W, wl.L, layer, wl.tri_start, stream)
+
+    tri_f, causal_f = tile_flop(wl, False, W), tile_flop(wl, True)
+
+    for _ in range(args.warmup):
+        layer_call(tri_layer)
+        layer_call(causal_layer)
+    torch.cuda.synchronize()
+    if tm.tm_get_device_status(stream) != tm.TM_OK:
+        raise RuntimeError("device status not ok after warm-up")
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    for s in range(args.steps):
+        ev[s][0].record(stream)
+        layer_call(tri_layer)
+        ev[s][1].record(stream)
+        layer_call(causal_layer)
+        ev[s][2].record(stream)
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    status = tm.tm_get_device_status(stream)
+    tri_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(args.steps)]
+    cau_ms = [ev[s][1].elapsed_time(ev[s][2]) for s in range(args.steps)]
+    total_ms = ev[0][0].elapsed_time(ev[-1][2])
+    tri_sum = sum(tri_ms)
+
+    # end to end through the same call: pinned host -> device, layer, device -> host
+    e2e_steps = max(1, min(args.steps, 3))
+    ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(e2e_steps)]
+    for s in range(e2e_steps):
+        ee[s][0].record(stream)
+        for d, h in ((dq, hq), (dk, hk), (dv, hv)):
+            d.view(torch.int16).copy_(h, non_blocking=True)
+        layer_call(tri_layer)
+        ho.copy_(do.view(torch.int16), non_blocking=True)
+        ee[s][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(ee[s][0].elapsed_time(ee[s][1]) for s in range(e2e_steps)) / e2e_steps
+
+    if ws > 1:
+        t = torch.tensor([total_ms, tri_sum, e2e_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, tri_sum, e2e_ms = t.tolist()
+
+    peaks = load_peaks()
+    tri_avg = tri_sum / args.steps
+    achieved = tri_f / (tri_avg * 1e-3) / 1e12
+    value = ws * args.steps * tri_f / (tri_sum * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "N": wl.N,
+                   "D": wl.D, "S": wl.S, "W": W, "L": wl.L, "tri_start": wl.tri_start,
+                   "step": "triangle layer + causal layer via tm_trianglemix_attn_fwd",
+                   "l2": "inputs larger than L2 (q alone is %.2f GB)" % (dq.numel() * 2 / 1e9),
+                   "parallelism": "replicas" if ws > 1 else "single"},
+        "triangle_ms": tri_avg,
+        "triangle_ms_p10_p90": [float(np.percentile(tri_ms, 10)), float(np.percentile(tri_ms, 90))],
+        "causal_ms": sum(cau_ms) / args.steps,
+        "causal_tflops": causal_f / (sum(cau_ms) / args.steps * 1e-3) / 1e12,
+        "speedup_vs_causal": (sum(cau_ms) / args.steps) / tri_avg,
+        "kept_tile_tflop": tri_f / 1e12,
+        "kept_pair_tflops": (tm.tm_triangle_kept_pairs(wl.N, wl.S, W, wl.L) * wl.B * wl.Hq * 4.0
+                             * wl.D) / (tri_avg * 1e-3) / 1e12,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["sustained"],
+                     "unit": "TFLOP/s", "frac": achieved / peaks["sustained"],
+                     "peak_kind": f"bf16 dense, {peaks['source']} sustained (kernel runs inside "
+                                  "a long step after the causal layer)",
+                     "frac_of_burst": achieved / peaks["burst"],
+                     "traffic": TRAFFIC.get(kernel_source_hash())},
+        "e2e": {"value": ws * tri_f / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": int((dq.numel() + dk.numel() + dv.numel()) * 2),
+                "d2h_bytes_per_step": int(do.numel() * 2),
+                "what": "pinned host q,k,v -> device, triangle layer, output -> pinned host"},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+        "device_status": tm.status_string(status),
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        dt, equiv, cores, desc = oracle_sample(wl, W, args.cpu_rows, 7, host_np)
+        line["cpu_baseline"] = {"value": equiv / dt / 1e12, "unit": UNIT, "cores": cores,
+                                "kind": "oracle", "sample": desc, "seconds": dt}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0 if status == tm.TM_OK else 1
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="llama3-8b-128k", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--window", type=int, default=0, help="override W of the workload")
+    ap.add_argument("--cpu-rows", type=int, default=24, help="oracle rows for cpu_baseline")
+    ap.add_argument("--ref-rows", type=int, default=8, help="oracle rows per reference step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps, always
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,155 @@
+/*
+ * tm.h - C ABI of the TriangleMix prefill-attention library for NVIDIA B200 (sm_100a).
+ *
+ * TriangleMix (He Zhiyuan's blog post "TriangleMix", sections 介绍 and 性能;
+ * the 36kr interview with Yang Yuqing, lead paragraphs) runs dense causal
+ * attention in the shallow layers of a model and a static "triangle" pattern
+ * in the deep layers, from layer index tri_start on. In the triangle pattern
+ * query row i attends key j (j <= i) only if
+ *     j < S          (one of the first S "sink" tokens of the streaming region),
+ *  or i - j < W      (one of the W most recent positions, i itself included),
+ *  or i >= N - L     (i is one of the last L queries: the "last Q-K" region,
+ *                     which sees every causal key).
+ * Everything else (the "middle Q-K" region) is skipped. The result is exact
+ * masked softmax attention over that key set:
+ *     o_i = sum_{j in K_i} softmax_j(scale * q_i . k_j) v_j.
+ *
+ * Tensor layout (all entry points): bf16, contiguous,
+ *     q, o : [B, N, Hq,  D]      k, v : [B, N, Hkv, D]
+ * Query head hq reads kv head hq / (Hq / Hkv) (consecutive q heads share a kv
+ * head). D must be 64 or 128. RoPE, if any, is applied by the caller.
+ *
+ * Ownership and threading:
+ *   - q, k, v, o are DEVICE pointers owned by the caller, 16-byte aligned;
+ *     o must not overlap q, k or v. The library allocates no device memory
+ *     in any call and keeps no per-call state.
+ *   - `stream` is a cudaStream_t (CUstream) handle passed as void*; NULL is
+ *     the legacy default stream. Work is enqueued asynchronously on it and
+ *     the call returns without synchronising.
+ *   - Calls are thread-safe. No C++ exception crosses this interface.
+ *
+ * Errors: every entry point returns a tm_status. Argument errors are reported
+ * synchronously, before anything is enqueued. TM_ERR_CUDA means a CUDA call
+ * failed (launch or driver). A kernel that gives up waiting on one of its own
+ * pipeline barriers (a bounded wait, about two seconds) records
+ * TM_ERR_TIMEOUT in a device status word, finishes cleanly and leaves the
+ * context usable; tm_get_device_status() reports it.
+ */
+#ifndef TM_H_
+#define TM_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(_WIN32)
+#define TM_API __declspec(dllexport)
+#else
+#define TM_API __attribute__((visibility("default")))
+#endif
+
+typedef enum {
+  TM_OK = 0,
+  TM_ERR_INVALID_ARG = -1,  /* null/misaligned/overlapping pointer, bad size or pattern */
+  TM_ERR_UNSUPPORTED = -2,  /* valid but not built: D not in {64,128}, not an sm_100 device */
+  TM_ERR_CUDA = -3,         /* a CUDA runtime/driver call failed */
+  TM_ERR_TIMEOUT = -4       /* a kernel gave up on a pipeline wait (device status) */
+} tm_status;
+
+/* Tile shape of the kernels (query rows x key columns per tile). */
+#define TM_BLOCK_M 128
+#define TM_BLOCK_N 128
+
+/*
+ * Dense causal attention, keep(i, j) = j <= i. This is the "full attention"
+ * the TriangleMix pages compare against (blog post, section 速度).
+ * scale: the softmax scale applied to q.k (commonly 1/sqrt(D)); must be finite.
+ */
+TM_API int tm_causal_attn_fwd(const void* q, const void* k, const void* v, void* o, int B,
+                              int Hq, int Hkv, int N, int D, float scale, void* stream);
+
+/*
+ * Triangle attention with sink count S, window W and last-query count L
+ * (blog post, section 介绍 and the "Middle Q-K" figure discussion in 缘由;
+ * 36kr interview, lead paragraph on the streaming and last Q-K regions).
+ * S >= 0, L >= 0, W >= 1; S and L larger than N act as N. L = N, or S + W >= N,
+ * gives the same result as tm_causal_attn_fwd.
+ */
+TM_API int tm_triangle_attn_fwd(const void* q, const void* k, const void* v, void* o, int B,
+                                int Hq, int Hkv, int N, int D, float scale, int S, int W, int L,
+                                void* stream);
+
+/*
+ * Layer schedule (blog post, section 性能: layers before the chosen start run
+ * full attention, the rest run triangle attention; 36kr interview:
+ * "L_tri_start = 12"). layer and tri_start are 0-based: layer < tri_start runs
+ * tm_causal_attn_fwd, layer >= tri_start runs tm_triangle_attn_fwd with
+ * (S, W, L). layer >= 0 and tri_start >= 0 are required; S, W, L are validated
+ * only when the triangle kernel is chosen.
+ */
+TM_API int tm_trianglemix_attn_fwd(const void* q, const void* k, const void* v, void* o, int B,
+                                   int Hq, int Hkv, int N, int D, float scale, int S, int W,
+                                   int L, int layer, int tri_start, void* stream);
+
+/*
+ * Number of kept (i, j) pairs of one (batch, head) of the triangle pattern:
+ * sum over rows of min(i+1, W) + max(0, min(S, i+1-W)) for i < N-L and i+1
+ * otherwise. Host only. Returns -1 on a bad argument.
+ */
+TM_API long long tm_triangle_kept_pairs(int N, int S, int W, int L);
+
+/*
+ * Number of TM_BLOCK_M x TM_BLOCK_N tiles the kernel visits for one
+ * (batch, head): tiles holding at least one kept pair. causal != 0 counts
+ * the causal pattern (S, W, L ignored). Host only. -1 on a bad argument.
+ */
+TM_API long long tm_kept_tiles(int N, int causal, int S, int W, int L);
+
+/*
+ * Host export of the static tile list the kernels derive on the device, at
+ * tile shape (BM, BN) (the kernels use TM_BLOCK_M x TM_BLOCK_N). One record is
+ * three ints (qb, kb, full): q-block, k-block, and 1 if every pair of the
+ * tile's existing rows and columns is kept (no mask needed), else 0. Records
+ * are ordered by qb ascending, then kb ascending; tiles without a kept pair
+ * are absent. out: HOST buffer of 3*cap ints (may be NULL when cap = 0);
+ * *count receives the total number of records even when it exceeds cap.
+ * tm_triangle_tile_list is the triangle pattern; tm_tile_list selects causal.
+ */
+TM_API int tm_triangle_tile_list(int N, int S, int W, int L, int BM, int BN, int* out,
+                                 long long cap, long long* count);
+TM_API int tm_tile_list(int N, int causal, int S, int W, int L, int BM, int BN, int* out,
+                        long long cap, long long* count);
+
+/*
+ * Device dump of the same list, produced by the kernels' own device code at
+ * TM_BLOCK_M x TM_BLOCK_N. out_dev: DEVICE buffer of 3*cap ints; *count
+ * (host) receives the record total; records beyond cap are not written.
+ * Asynchronous on `stream`.
+ */
+TM_API int tm_debug_dump_tiles(int N, int causal, int S, int W, int L, int* out_dev,
+                               long long cap, long long* count, void* stream);
+
+/*
+ * Building-block check of the tensor-core path on one 128-row tile:
+ * s_out[128*128] = q k^T (fp32) and o_out[128*D] = bf16(q k^T) v (fp32), with
+ * q, k, v bf16 [128, D] DEVICE pointers and s_out, o_out fp32 DEVICE pointers.
+ * Asynchronous on `stream`.
+ */
+TM_API int tm_debug_mma_probe(const void* q, const void* k, const void* v, float* s_out,
+                              float* o_out, int D, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word of the
+ * current device: TM_OK, or TM_ERR_TIMEOUT if a kernel gave up on a wait
+ * since the last call. TM_ERR_CUDA if the synchronisation itself failed.
+ */
+TM_API int tm_get_device_status(void* stream);
+
+/* Static string for a status code; never NULL. */
+TM_API const char* tm_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TM_H_ */

@@ -1,0 +1,202 @@
+"""TriangleMix prefill attention on NVIDIA B200 (sm_100a).
+
+Python binding of ``libtm.so`` (C ABI in ``include/tm.h``). The functions named
+``tm_*`` take the C ABI's arguments one for one; tensors may be passed as
+torch tensors (their ``data_ptr()`` is used) or as raw device addresses.
+This module only marshals arguments: every step of the attention runs in the
+library's CUDA kernels. PyTorch provides device memory and streams.
+
+If the library has not been built, every call raises; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtm.so")
+
+TM_OK, TM_ERR_INVALID_ARG, TM_ERR_UNSUPPORTED, TM_ERR_CUDA, TM_ERR_TIMEOUT = 0, -1, -2, -3, -4
+TM_BLOCK_M = TM_BLOCK_N = 128
+
+EXPORTED = (
+    "tm_causal_attn_fwd", "tm_triangle_attn_fwd", "tm_trianglemix_attn_fwd",
+    "tm_triangle_kept_pairs", "tm_kept_tiles", "tm_triangle_tile_list", "tm_tile_list",
+    "tm_debug_dump_tiles", "tm_debug_mma_probe", "tm_get_device_status", "tm_status_string",
+)
+
+
+class TmError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {status} ({status_string(status)})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded ``libtm.so``; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing; build it with "
+                "`python -m long_context_prefill_trianglemix_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, ci, cf, cll = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_longlong
+        sig = {
+            "tm_causal_attn_fwd": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp]),
+            "tm_triangle_attn_fwd": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci, ci, vp]),
+            "tm_trianglemix_attn_fwd": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci, ci,
+                                             ci, ci, vp]),
+            "tm_triangle_kept_pairs": (cll, [ci, ci, ci, ci]),
+            "tm_kept_tiles": (cll, [ci, ci, ci, ci, ci]),
+            "tm_triangle_tile_list": (ci, [ci, ci, ci, ci, ci, ci, vp, cll,
+                                           ctypes.POINTER(cll)]),
+            "tm_tile_list": (ci, [ci, ci, ci, ci, ci, ci, ci, vp, cll, ctypes.POINTER(cll)]),
+            "tm_debug_dump_tiles": (ci, [ci, ci, ci, ci, ci, vp, cll, ctypes.POINTER(cll), vp]),
+            "tm_debug_mma_probe": (ci, [vp, vp, vp, vp, vp, ci, vp]),
+            "tm_get_device_status": (ci, [vp]),
+            "tm_status_string": (ctypes.c_char_p, [ci]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype, f.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().tm_status_string(int(status)).decode()
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if hasattr(x, "data_ptr"):
+        return x.data_ptr()
+    return int(x)
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if hasattr(s, "cuda_stream"):
+        return s.cuda_stream
+    return int(s)
+
+
+def _check(fn: str, rc: int) -> int:
+    if rc != TM_OK:
+        raise TmError(fn, rc)
+    return rc
+
+
+# ----------------------------------------------------------------------- C ABI, one for one
+
+def tm_causal_attn_fwd(q, k, v, o, B, Hq, Hkv, N, D, scale, stream=None):
+    return _check("tm_causal_attn_fwd", lib().tm_causal_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, Hkv, N, D, scale, _stream(stream)))
+
+
+def tm_triangle_attn_fwd(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L, stream=None):
+    return _check("tm_triangle_attn_fwd", lib().tm_triangle_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, Hkv, N, D, scale, S, W, L, _stream(stream)))
+
+
+def tm_trianglemix_attn_fwd(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L, layer, tri_start,
+                            stream=None):
+    return _check("tm_trianglemix_attn_fwd", lib().tm_trianglemix_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, Hkv, N, D, scale, S, W, L, layer, tri_start,
+        _stream(stream)))
+
+
+def tm_triangle_kept_pairs(N, S, W, L) -> int:
+    return int(lib().tm_triangle_kept_pairs(N, S, W, L))
+
+
+def tm_kept_tiles(N, causal, S, W, L) -> int:
+    return int(lib().tm_kept_tiles(N, int(causal), S, W, L))
+
+
+def tm_tile_list(N, causal, S, W, L, BM=TM_BLOCK_M, BN=TM_BLOCK_N) -> np.ndarray:
+    """(qb, kb, full) records of the static tile list, as an int32 [n, 3] array."""
+    cnt = ctypes.c_longlong(0)
+    _check("tm_tile_list", lib().tm_tile_list(N, int(causal), S, W, L, BM, BN, None, 0,
+                                              ctypes.byref(cnt)))
+    out = np.zeros((max(cnt.value, 1), 3), np.int32)
+    _check("tm_tile_list", lib().tm_tile_list(N, int(causal), S, W, L, BM, BN,
+                                              out.ctypes.data, cnt.value, ctypes.byref(cnt)))
+    return out[: cnt.value]
+
+
+def tm_triangle_tile_list(N, S, W, L, BM=TM_BLOCK_M, BN=TM_BLOCK_N) -> np.ndarray:
+    cnt = ctypes.c_longlong(0)
+    _check("tm_triangle_tile_list", lib().tm_triangle_tile_list(N, S, W, L, BM, BN, None, 0,
+                                                                ctypes.byref(cnt)))
+    out = np.zeros((max(cnt.value, 1), 3), np.int32)
+    _check("tm_triangle_tile_list", lib().tm_triangle_tile_list(
+        N, S, W, L, BM, BN, out.ctypes.data, cnt.value, ctypes.byref(cnt)))
+    return out[: cnt.value]
+
+
+def tm_debug_dump_tiles(N, causal, S, W, L, out_dev, cap, stream=None) -> int:
+    cnt = ctypes.c_longlong(0)
+    _check("tm_debug_dump_tiles", lib().tm_debug_dump_tiles(
+        N, int(causal), S, W, L, _ptr(out_dev), cap, ctypes.byref(cnt), _stream(stream)))
+    return cnt.value
+
+
+def tm_debug_mma_probe(q, k, v, s_out, o_out, D, stream=None):
+    return _check("tm_debug_mma_probe", lib().tm_debug_mma_probe(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(s_out), _ptr(o_out), D, _stream(stream)))
+
+
+def tm_get_device_status(stream=None) -> int:
+    return int(lib().tm_get_device_status(_stream(stream)))
+
+
+# ----------------------------------------------------------------------- torch conveniences
+
+def _shapes(q, k):
+    B, N, Hq, D = q.shape
+    Hkv = k.shape[2]
+    return B, N, Hq, Hkv, D
+
+
+def _out(q, out):
+    import torch
+    return torch.empty_like(q) if out is None else out
+
+
+def causal_attention(q, k, v, scale=None, out=None, stream=None):
+    """Dense causal attention of bf16 CUDA tensors q [B,N,Hq,D], k/v [B,N,Hkv,D]."""
+    B, N, Hq, Hkv, D = _shapes(q, k)
+    o = _out(q, out)
+    tm_causal_attn_fwd(q, k, v, o, B, Hq, Hkv, N, D,
+                       1.0 / math.sqrt(D) if scale is None else scale, stream)
+    return o
+
+
+def triangle_attention(q, k, v, S, W, L, scale=None, out=None, stream=None):
+    """Triangle attention (sinks S, window W, last L rows) of bf16 CUDA tensors."""
+    B, N, Hq, Hkv, D = _shapes(q, k)
+    o = _out(q, out)
+    tm_triangle_attn_fwd(q, k, v, o, B, Hq, Hkv, N, D,
+                         1.0 / math.sqrt(D) if scale is None else scale, S, W, L, stream)
+    return o
+
+
+def trianglemix_attention(q, k, v, S, W, L, layer, tri_start, scale=None, out=None, stream=None):
+    """One layer of the TriangleMix schedule: causal below tri_start, triangle from it on."""
+    B, N, Hq, Hkv, D = _shapes(q, k)
+    o = _out(q, out)
+    tm_trianglemix_attn_fwd(q, k, v, o, B, Hq, Hkv, N, D,
+                            1.0 / math.sqrt(D) if scale is None else scale, S, W, L, layer,
+                            tri_start, stream)
+    return o

@@ -1,0 +1,170 @@
+// C ABI of the library (declared in include/tm.h): argument validation, the
+// layer schedule, host exports of the static tile list, and status handling.
+// All device work is delegated to tm_attn.cu.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "tm.h"
+#include "tm_internal.h"
+#include "tm_tiles.cuh"
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, long long abytes, const void* b, long long bbytes) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + static_cast<uintptr_t>(bbytes) && b0 < a0 + static_cast<uintptr_t>(abytes);
+}
+
+int validate_common(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv,
+                    int N, int D, float scale) {
+  if (!q || !k || !v || !o) return TM_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || D < 1) return TM_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return TM_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return TM_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return TM_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return TM_ERR_INVALID_ARG;
+  // sizes must stay inside the 32-bit indices used for rows and work items
+  const long long rows = static_cast<long long>(B) * N;
+  if (rows > (1LL << 31) - 1 || static_cast<long long>(N) * Hq > (1LL << 31) - 1)
+    return TM_ERR_INVALID_ARG;
+  const long long nqb = (N + TM_BLOCK_M - 1) / TM_BLOCK_M;
+  if (nqb * B * Hkv * ((Hq / Hkv + 1) / 2) > (1LL << 31) - 1) return TM_ERR_INVALID_ARG;
+  const long long qbytes = rows * Hq * D * 2, kvbytes = rows * Hkv * D * 2;
+  if (overlaps(o, qbytes, q, qbytes) || overlaps(o, qbytes, k, kvbytes) ||
+      overlaps(o, qbytes, v, kvbytes))
+    return TM_ERR_INVALID_ARG;
+  return TM_OK;
+}
+
+int validate_pattern(int S, int W, int L) {
+  if (S < 0 || L < 0 || W < 1) return TM_ERR_INVALID_ARG;
+  return TM_OK;
+}
+
+int run(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv, int N, int D,
+        float scale, const trimix::Pattern& pat, void* stream) {
+  trimix::LaunchArgs a;
+  a.q = q; a.k = k; a.v = v; a.o = o;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.N = N; a.D = D;
+  a.scale = scale;
+  a.pat = pat;
+  a.stream = stream;
+  return trimix::launch_attention(a);
+}
+
+}  // namespace
+
+extern "C" {
+
+TM_API int tm_causal_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int Hq,
+                              int Hkv, int N, int D, float scale, void* stream) {
+  if (int rc = validate_common(q, k, v, o, B, Hq, Hkv, N, D, scale)) return rc;
+  return run(q, k, v, o, B, Hq, Hkv, N, D, scale, trimix::make_pattern(N, 1, 0, 1, 0), stream);
+}
+
+TM_API int tm_triangle_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int Hq,
+                                int Hkv, int N, int D, float scale, int S, int W, int L,
+                                void* stream) {
+  if (int rc = validate_common(q, k, v, o, B, Hq, Hkv, N, D, scale)) return rc;
+  if (int rc = validate_pattern(S, W, L)) return rc;
+  return run(q, k, v, o, B, Hq, Hkv, N, D, scale, trimix::make_pattern(N, 0, S, W, L), stream);
+}
+
+TM_API int tm_trianglemix_attn_fwd(const void* q, const void* k, const void* v, void* o, int B,
+                                   int Hq, int Hkv, int N, int D, float scale, int S, int W, int L,
+                                   int layer, int tri_start, void* stream) {
+  if (layer < 0 || tri_start < 0) return TM_ERR_INVALID_ARG;
+  if (layer < tri_start) return tm_causal_attn_fwd(q, k, v, o, B, Hq, Hkv, N, D, scale, stream);
+  return tm_triangle_attn_fwd(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L, stream);
+}
+
+TM_API long long tm_triangle_kept_pairs(int N, int S, int W, int L) {
+  if (N < 1 || validate_pattern(S, W, L)) return -1;
+  const trimix::Pattern p = trimix::make_pattern(N, 0, S, W, L);
+  long long total = 0;
+  for (long long i = 0; i < N; ++i) {
+    if (i >= p.N - p.L) {
+      total += i + 1;
+    } else {
+      const long long w = i + 1 < p.W ? i + 1 : p.W;
+      long long extra = i + 1 - p.W;
+      if (extra > p.S) extra = p.S;
+      total += w + (extra > 0 ? extra : 0);
+    }
+  }
+  return total;
+}
+
+TM_API long long tm_kept_tiles(int N, int causal, int S, int W, int L) {
+  if (N < 1 || (!causal && validate_pattern(S, W, L))) return -1;
+  const trimix::Pattern p = trimix::make_pattern(N, causal, S, W, L);
+  const int nqb = (N + TM_BLOCK_M - 1) / TM_BLOCK_M;
+  long long n = 0;
+  for (int qb = 0; qb < nqb; ++qb) n += trimix::block_tiles(p, qb, TM_BLOCK_M, TM_BLOCK_N).count();
+  return n;
+}
+
+TM_API int tm_tile_list(int N, int causal, int S, int W, int L, int BM, int BN, int* out,
+                        long long cap, long long* count) {
+  if (N < 1 || BM < 1 || BN < 1 || cap < 0 || !count || (cap > 0 && !out))
+    return TM_ERR_INVALID_ARG;
+  if (!causal && validate_pattern(S, W, L)) return TM_ERR_INVALID_ARG;
+  const trimix::Pattern p = trimix::make_pattern(N, causal, S, W, L);
+  const int nqb = (N + BM - 1) / BM;
+  long long n = 0;
+  for (int qb = 0; qb < nqb; ++qb) {
+    const trimix::BlockTiles bt = trimix::block_tiles(p, qb, BM, BN);
+    for (int t = 0; t < bt.count(); ++t, ++n) {
+      if (n >= cap) continue;
+      const int kb = bt.kb(t);
+      out[3 * n + 0] = qb;
+      out[3 * n + 1] = kb;
+      out[3 * n + 2] = trimix::tile_full(p, qb, kb, BM, BN);
+    }
+  }
+  *count = n;
+  return TM_OK;
+}
+
+TM_API int tm_triangle_tile_list(int N, int S, int W, int L, int BM, int BN, int* out,
+                                 long long cap, long long* count) {
+  return tm_tile_list(N, 0, S, W, L, BM, BN, out, cap, count);
+}
+
+TM_API int tm_debug_dump_tiles(int N, int causal, int S, int W, int L, int* out_dev, long long cap,
+                               long long* count, void* stream) {
+  if (N < 1 || cap < 0 || !count || (cap > 0 && !out_dev) || !aligned16(out_dev))
+    return TM_ERR_INVALID_ARG;
+  if (!causal && validate_pattern(S, W, L)) return TM_ERR_INVALID_ARG;
+  const long long n = tm_kept_tiles(N, causal, S, W, L);
+  if (n < 0) return TM_ERR_INVALID_ARG;
+  *count = n;
+  return trimix::launch_dump_tiles(trimix::make_pattern(N, causal, S, W, L), out_dev, cap, stream);
+}
+
+TM_API int tm_debug_mma_probe(const void* q, const void* k, const void* v, float* s_out,
+                              float* o_out, int D, void* stream) {
+  if (!q || !k || !v || !s_out || !o_out) return TM_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return TM_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return TM_ERR_UNSUPPORTED;
+  return trimix::launch_mma_probe(q, k, v, s_out, o_out, D, stream);
+}
+
+TM_API int tm_get_device_status(void* stream) { return trimix::read_and_clear_device_status(stream); }
+
+TM_API const char* tm_status_string(int status) {
+  switch (status) {
+    case TM_OK: return "ok";
+    case TM_ERR_INVALID_ARG: return "invalid argument";
+    case TM_ERR_UNSUPPORTED: return "unsupported configuration or device";
+    case TM_ERR_CUDA: return "CUDA error";
+    case TM_ERR_TIMEOUT: return "kernel gave up on a pipeline wait";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

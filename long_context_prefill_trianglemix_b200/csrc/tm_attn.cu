@@ -1,0 +1,835 @@
+// TriangleMix prefill attention for sm_100a: one persistent, warp-specialised
+// kernel template for the dense causal pattern and the static triangle pattern.
+//
+// What is computed is exact masked softmax attention over the kept key set of
+// each query row (TriangleMix blog post, sections 介绍 and 缘由; 36kr interview,
+// lead paragraphs): the triangle keeps the first S sink keys, the W most recent
+// keys and, for the last L query rows, every causal key.
+//
+// CTA layout (384 threads, one CTA per SM, persistent):
+//   warps 0-3  softmax warpgroup 0: rows of Q tile 0 (TMEM lanes 0..127)
+//   warps 4-7  softmax warpgroup 1: rows of Q tile 1
+//   warp  8    TMA producer (one elected thread): Q tiles, then K/V tiles
+//   warp  9    tcgen05 issuer (one elected thread) and TMEM owner
+//   warps 10-11 idle (they complete the third warpgroup for setmaxnreg)
+// The kernel is launched at 168 registers per thread (384 x 168 = 64512);
+// the third warpgroup drops to 88 and the softmax warpgroups rise to 208
+// (2 x 128 x 208 + 128 x 88 = 64512), so the row of 128 scores stays in
+// registers. The host refuses to launch a build whose register count differs.
+// A work item is (batch, kv head, pair of q heads of that kv head's group,
+// q-block): both Q tiles read the same K/V stream, which is loaded once. Only
+// the kept k-blocks of the q-block are visited (tm_tiles.cuh); elementwise
+// masking runs only on the tiles that need it.
+//
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).
+// P (bf16) overwrites the first 64 columns of its S tile once S has been read
+// into registers, and feeds the P.V MMA directly from TMEM.
+//
+// MMA issue order per item (K_t, V_t are ring slots, in load order):
+//   S0=Q0.K0  S1=Q1.K0 | for t: O0+=P0.V_t  S0=Q0.K_{t+1}  O1+=P1.V_t  S1=Q1.K_{t+1}
+// so one softmax warpgroup works while the tensor core runs the other's MMAs.
+//
+// Every wait is bounded (about two seconds). On expiry the kernel records a
+// timeout in g_status, every role leaves its loop, in-flight copies and MMAs
+// are drained with bounded waits, TMEM is freed and the CTA exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <mutex>
+#include <vector>
+
+#include "tm.h"
+#include "tm_internal.h"
+#include "tm_sm100.cuh"
+#include "tm_tiles.cuh"
+
+namespace trimix {
+
+using namespace sm100;
+
+__device__ int g_status = 0;
+__device__ int g_status_where = 0;
+
+constexpr int BM = TM_BLOCK_M;
+constexpr int BN = TM_BLOCK_N;
+static_assert(BM == 128 && BN == 128, "tile shape is fixed by the TMEM layout");
+constexpr int kThreads = 384;
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 208;
+constexpr int kSideRegs = 88;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kSideRegs == kThreads * kLaunchRegs,
+              "register split must use exactly the registers the CTA is launched with");
+constexpr int kWarpTma = 8;
+constexpr int kWarpMma = 9;
+constexpr int kMaxCtas = 192;
+constexpr uint32_t kTmemCols = 512;
+// Keep a stale running max until the true max exceeds it by 2^8: p stays <= 256
+// in fp32/bf16, and the O rescale (a TMEM round trip) becomes rare.
+constexpr float kRescaleThreshold = 8.0f;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr uint64_t kDrainLimitNs = 100000000ull;
+
+// Where a wait gave up (recorded with the timeout, for diagnosis).
+enum WaitSite : int {
+  kSiteQEmpty = 1, kSiteKvEmpty, kSiteQFull, kSiteKvFull, kSiteOEmpty, kSitePFull,
+  kSiteSFull, kSiteOFull, kSiteProbe
+};
+
+template <int D>
+struct Cfg {
+  static constexpr int kTileBytes = BM * D * 2;  // one Q, K or V tile (BM == BN)
+  static constexpr int kPanelBytes = BM * 64 * 2; // one 128-byte-wide swizzle panel
+  static constexpr int kPanels = D / 64;
+  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kRingOff = 2 * kTileBytes;
+  static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
+  static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // barriers + alignment slack
+  static constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128;
+  static constexpr uint32_t kTmemO0 = 256, kTmemO1 = 256 + D;
+  static constexpr uint32_t kIdescS = idesc_bf16_f32(BM, BN, 0, 0);  // Q, K both K-major
+  static constexpr uint32_t kIdescO = idesc_bf16_f32(BM, D, 0, 1);   // V is MN-major
+};
+
+template <int NST>
+struct Bars {
+  uint64_t q_full, q_empty;
+  uint64_t kv_full[NST], kv_empty[NST];
+  uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct AttnParams {
+  int B, Hq, Hkv, N, G, npairs, nqb, units;
+  Pattern pat;
+  float sl2;  // softmax scale * log2(e)
+  __nv_bfloat16* o;
+  int cta_begin[kMaxCtas + 1];
+};
+
+struct Item {
+  int b, g, qb, h0, v1;
+};
+
+__host__ __device__ __forceinline__ Item decode_item(int B, int Hkv, int G, int npairs, int nqb,
+                                                     int units, int item) {
+  (void)B;
+  Item it;
+  const int qi = item / units;
+  const int u = item - qi * units;
+  it.qb = nqb - 1 - qi;  // longest q-blocks first
+  const int pr = u % npairs;
+  const int gb = u / npairs;
+  it.g = gb % Hkv;
+  it.b = gb / Hkv;
+  it.h0 = it.g * G + 2 * pr;
+  it.v1 = (2 * pr + 1 < G) ? 1 : 0;
+  return it;
+}
+
+__device__ __forceinline__ void record_timeout(int site) {
+  if (atomicCAS(&g_status, kDevOk, kDevTimeout) == kDevOk) g_status_where = site;
+}
+
+// Bounded mbarrier wait. false = gave up (timeout here, or abort seen).
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                      int site) {
+  const uint32_t a = smem_addr(bar);
+  if (mbar_try_wait(a, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(a, parity)) return true;
+    if ((it & 31u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        record_timeout(site);
+        return false;
+      }
+    }
+  }
+}
+
+// Short wait used only while draining after an abort.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_addr(bar);
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(a, parity)) {
+    if (globaltimer_ns() - t0 > kDrainLimitNs) return;
+  }
+}
+
+// ------------------------------------------------------------------ MMA helpers
+
+// S[128 x 128] = Q[128 x D] . K[128 x D]^T; both tiles K-major, 128B-swizzled,
+// stored as D/64 panels of 128 rows x 128 bytes.
+template <int D>
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_base, uint32_t k_base) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * Cfg<D>::kPanelBytes + (kk & 3) * 32;
+    mma_ss(d_tmem, smem_desc_sw128(q_base + off, 16, 1024), smem_desc_sw128(k_base + off, 16, 1024),
+           Cfg<D>::kIdescS, kk > 0 ? 1u : 0u);
+  }
+}
+
+// O[128 x D] (+)= P[128 x 128] (bf16 in TMEM, 2 per column) . V[128 x D];
+// V is MN-major (D contiguous per key row): 16 keys per step = 16 rows.
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_base,
+                                         uint32_t accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < BN / 16; ++kk) {
+    mma_ts(d_tmem, p_tmem + kk * 8, smem_desc_sw128(v_base + kk * 16 * 128, Cfg<D>::kPanelBytes, 1024),
+           Cfg<D>::kIdescO, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+// Bits [0, n) of a 32-bit word, n clamped to [0, 32].
+__device__ __forceinline__ uint32_t range_bits(int n) {
+  n = n < 0 ? 0 : (n > 32 ? 32 : n);
+  return n == 32 ? 0xFFFFFFFFu : ((1u << n) - 1u);
+}
+
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                 "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                 "+r"(r[30]), "+r"(r[31]));
+}
+
+// ------------------------------------------------------------------ roles
+
+template <int D>
+__device__ __forceinline__ void producer_role(const AttnParams& p, Bars<Cfg<D>::kStages>* bars,
+                                              uint8_t* smem, const CUtensorMap* tq,
+                                              const CUtensorMap* tk, const CUtensorMap* tv) {
+  constexpr int NST = Cfg<D>::kStages;
+  volatile int* abort_flag = &bars->abort_flag;
+  const uint32_t q0 = smem_addr(smem);
+  const uint32_t ring = smem_addr(smem + Cfg<D>::kRingOff);
+  uint32_t kv_cnt = 0, it_cnt = 0;
+  bool ok = true;
+  for (int item = p.cta_begin[blockIdx.x]; ok && item < p.cta_begin[blockIdx.x + 1]; ++item) {
+    const Item it = decode_item(p.B, p.Hkv, p.G, p.npairs, p.nqb, p.units, item);
+    const BlockTiles bt = block_tiles(p.pat, it.qb, BM, BN);
+    if (!(ok = wait_bar(&bars->q_empty, (it_cnt & 1u) ^ 1u, abort_flag, kSiteQEmpty))) break;
+    mbar_arrive_expect_tx(&bars->q_full, (1 + it.v1) * Cfg<D>::kTileBytes);
+#pragma unroll
+    for (int pn = 0; pn < Cfg<D>::kPanels; ++pn) {
+      tma_load_4d(q0 + pn * Cfg<D>::kPanelBytes, tq, &bars->q_full, pn * 64, it.h0, it.qb * BM, it.b);
+      if (it.v1)
+        tma_load_4d(q0 + Cfg<D>::kTileBytes + pn * Cfg<D>::kPanelBytes, tq, &bars->q_full, pn * 64,
+                    it.h0 + 1, it.qb * BM, it.b);
+    }
+    ++it_cnt;
+    const int T = bt.count();
+    for (int t = 0; ok && t < T; ++t) {
+      const int kb = bt.kb(t);
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t st = kv_cnt % NST;
+        if (!(ok = wait_bar(&bars->kv_empty[st], ((kv_cnt / NST) & 1u) ^ 1u, abort_flag,
+                            kSiteKvEmpty)))
+          break;
+        mbar_arrive_expect_tx(&bars->kv_full[st], Cfg<D>::kTileBytes);
+#pragma unroll
+        for (int pn = 0; pn < Cfg<D>::kPanels; ++pn)
+          tma_load_4d(ring + st * Cfg<D>::kTileBytes + pn * Cfg<D>::kPanelBytes, which ? tv : tk,
+                      &bars->kv_full[st], pn * 64, it.g, kb * BN, it.b);
+        ++kv_cnt;
+      }
+    }
+  }
+  if (!ok) {  // let copies already in flight land before the CTA goes away
+    const uint32_t first = kv_cnt > (uint32_t)NST ? kv_cnt - NST : 0;
+    for (uint32_t idx = first; idx < kv_cnt; ++idx)
+      drain_wait(&bars->kv_full[idx % NST], (idx / NST) & 1u);
+    if (it_cnt) drain_wait(&bars->q_full, (it_cnt - 1) & 1u);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStages>* bars,
+                                         uint8_t* smem, uint32_t tmem_base) {
+  constexpr int NST = Cfg<D>::kStages;
+  volatile int* abort_flag = &bars->abort_flag;
+  const uint32_t q0 = smem_addr(smem), q1 = q0 + Cfg<D>::kTileBytes;
+  const uint32_t ring = smem_addr(smem + Cfg<D>::kRingOff);
+  const uint32_t tS0 = tmem_base + Cfg<D>::kTmemS0, tS1 = tmem_base + Cfg<D>::kTmemS1;
+  const uint32_t tO0 = tmem_base + Cfg<D>::kTmemO0, tO1 = tmem_base + Cfg<D>::kTmemO1;
+  uint32_t kv_cnt = 0, it_cnt = 0, pc0 = 0, pc1 = 0, oe0 = 0, oe1 = 0;
+  bool ok = true;
+#define TM_WAIT(bar, par, site)                                      \
+  if (!(ok = wait_bar((bar), (par), abort_flag, (site)))) break; \
+  tc_fence_after();
+  for (int item = p.cta_begin[blockIdx.x]; ok && item < p.cta_begin[blockIdx.x + 1]; ++item) {
+    const Item it = decode_item(p.B, p.Hkv, p.G, p.npairs, p.nqb, p.units, item);
+    const int T = block_tiles(p.pat, it.qb, BM, BN).count();
+    const bool v1 = it.v1 != 0;
+    TM_WAIT(&bars->q_full, it_cnt & 1u, kSiteQFull);
+    ++it_cnt;
+    uint32_t kst = kv_cnt % NST;
+    TM_WAIT(&bars->kv_full[kst], (kv_cnt / NST) & 1u, kSiteKvFull);
+    issue_qk<D>(tS0, q0, ring + kst * Cfg<D>::kTileBytes);
+    mma_commit(&bars->s_full[0]);
+    if (v1) {
+      issue_qk<D>(tS1, q1, ring + kst * Cfg<D>::kTileBytes);
+      mma_commit(&bars->s_full[1]);
+    }
+    if (T == 1) mma_commit(&bars->q_empty);
+    mma_commit(&bars->kv_empty[kst]);
+    ++kv_cnt;
+    for (int t = 0; t < T; ++t) {
+      const uint32_t vst = kv_cnt % NST;
+      TM_WAIT(&bars->kv_full[vst], (kv_cnt / NST) & 1u, kSiteKvFull);
+      if (t == 0) {
+        TM_WAIT(&bars->o_empty[0], (oe0 & 1u) ^ 1u, kSiteOEmpty);
+        ++oe0;
+      }
+      TM_WAIT(&bars->p_full[0], pc0 & 1u, kSitePFull);
+      ++pc0;
+      issue_pv<D>(tO0, tS0, ring + vst * Cfg<D>::kTileBytes, t > 0 ? 1u : 0u);
+      if (t == T - 1) mma_commit(&bars->o_full[0]);
+      if (t + 1 < T) {
+        const uint32_t kidx = kv_cnt + 1;
+        kst = kidx % NST;
+        TM_WAIT(&bars->kv_full[kst], (kidx / NST) & 1u, kSiteKvFull);
+        issue_qk<D>(tS0, q0, ring + kst * Cfg<D>::kTileBytes);
+        mma_commit(&bars->s_full[0]);
+        if (!v1 && t + 1 == T - 1) mma_commit(&bars->q_empty);
+      }
+      if (v1) {
+        if (t == 0) {
+          TM_WAIT(&bars->o_empty[1], (oe1 & 1u) ^ 1u, kSiteOEmpty);
+          ++oe1;
+        }
+        TM_WAIT(&bars->p_full[1], pc1 & 1u, kSitePFull);
+        ++pc1;
+        issue_pv<D>(tO1, tS1, ring + vst * Cfg<D>::kTileBytes, t > 0 ? 1u : 0u);
+        if (t == T - 1) mma_commit(&bars->o_full[1]);
+      }
+      mma_commit(&bars->kv_empty[vst]);  // V_t free once both P.V products are done
+      ++kv_cnt;
+      if (t + 1 < T) {
+        if (v1) {
+          issue_qk<D>(tS1, q1, ring + kst * Cfg<D>::kTileBytes);
+          mma_commit(&bars->s_full[1]);
+          if (t + 1 == T - 1) mma_commit(&bars->q_empty);
+        }
+        mma_commit(&bars->kv_empty[kst]);  // K_{t+1} free once both Q.K products are done
+        ++kv_cnt;
+      }
+    }
+  }
+#undef TM_WAIT
+  // Every MMA issued above must finish before TMEM is released.
+  mma_commit(&bars->mma_done);
+  drain_wait(&bars->mma_done, 0);
+}
+
+template <int D>
+__device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::kStages>* bars,
+                                             int wg, int wq, int lane, uint32_t tmem_base) {
+  volatile int* abort_flag = &bars->abort_flag;
+  const int r = wq * 32 + lane;  // row of the Q tile == TMEM lane
+  const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
+  const uint32_t tS = tmem_base + lane_addr + (wg ? Cfg<D>::kTmemS1 : Cfg<D>::kTmemS0);
+  const uint32_t tO = tmem_base + lane_addr + (wg ? Cfg<D>::kTmemO1 : Cfg<D>::kTmemO0);
+  const float sl2 = p.sl2;
+  const Pattern& pat = p.pat;
+  uint32_t s_cnt = 0, o_cnt = 0;
+  for (int item = p.cta_begin[blockIdx.x]; item < p.cta_begin[blockIdx.x + 1]; ++item) {
+    const Item it = decode_item(p.B, p.Hkv, p.G, p.npairs, p.nqb, p.units, item);
+    if (wg == 1 && !it.v1) continue;
+    const BlockTiles bt = block_tiles(pat, it.qb, BM, BN);
+    const int T = bt.count();
+    const int i = it.qb * BM + r;  // query row of this thread
+    // kept keys of row i: [0, sink_hi) U [band_lo, hi)
+    const int hi = imin(i, pat.N - 1) + 1;
+    const bool full_row = pat.causal || i >= pat.N - pat.L;
+    const int sink_hi = full_row ? hi : imin(pat.S, hi);
+    const int band_lo = full_row ? hi : imax(0, i - pat.W + 1);
+    float m_run = -INFINITY, l_run = 0.f;
+    for (int t = 0; t < T; ++t) {
+      const int kb = bt.kb(t);
+      const bool need_mask = tile_needs_mask(pat, it.qb, kb, BM, BN) != 0;
+      bool ok = wait_bar(&bars->s_full[wg], s_cnt & 1u, abort_flag, kSiteSFull);
+      ++s_cnt;
+      if (!__all_sync(0xffffffffu, ok)) return;
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, sr[c]);
+      tmem_wait_ld(sr[0]);
+      reg_fence(sr[1]);
+      reg_fence(sr[2]);
+      reg_fence(sr[3]);
+      if (need_mask) {
+        // keep bits of this row for the tile's 128 columns, then -inf elsewhere
+        const int c0 = kb * BN;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t keep = range_bits(sink_hi - c0 - 32 * c) |
+                                (range_bits(hi - c0 - 32 * c) & ~range_bits(band_lo - c0 - 32 * c));
+#pragma unroll
+          for (int x = 0; x < 32; ++x)
+            sr[c][x] = ((keep >> x) & 1u) ? sr[c][x] : 0xFF800000u;
+        }
+      }
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int x = 0; x < 32; ++x) s[32 * c + x] = __uint_as_float(sr[c][x]);
+      float mx = s[0];
+#pragma unroll
+      for (int x = 1; x < 128; ++x) mx = fmaxf(mx, s[x]);
+      const float m_new = fmaxf(m_run, mx * sl2);
+      const bool bump = m_new > m_run + kRescaleThreshold;
+      float alpha = 1.f;
+      if (bump) {
+        alpha = ex2(m_run - m_new);
+        m_run = m_new;
+      }
+      const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
+      float rs = 0.f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          const float a = ex2(fmaf(s[64 * h + 2 * x], sl2, neg_m));
+          const float b = ex2(fmaf(s[64 * h + 2 * x + 1], sl2, neg_m));
+          rs += a + b;
+          pk[x] = pack_bf16x2(a, b);
+        }
+        tmem_st32(tS + 32 * h, pk);
+      }
+      l_run = l_run * alpha + rs;
+      if (t > 0 && __any_sync(0xffffffffu, bump)) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t orr[32];
+          tmem_ld32(tO + 32 * c, orr);
+          tmem_wait_ld(orr);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) orr[x] = __float_as_uint(__uint_as_float(orr[x]) * alpha);
+          tmem_st32(tO + 32 * c, orr);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[wg]);
+    }
+    // epilogue: O / l -> bf16 -> global
+    bool ok = wait_bar(&bars->o_full[wg], o_cnt & 1u, abort_flag, kSiteOFull);
+    ++o_cnt;
+    if (!__all_sync(0xffffffffu, ok)) return;
+    tc_fence_after();
+    uint32_t orr[D / 32][32];
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + 32 * c, orr[c]);
+    tmem_wait_ld(orr[0]);
+#pragma unroll
+    for (int c = 1; c < D / 32; ++c) reg_fence(orr[c]);
+    tc_fence_before();
+    mbar_arrive(&bars->o_empty[wg]);
+    const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+    if (i < pat.N) {
+      __nv_bfloat16* dst =
+          p.o + ((static_cast<size_t>(it.b) * pat.N + i) * p.Hq + (it.h0 + wg)) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x)
+          pk[x] = pack_bf16x2(__uint_as_float(orr[c][2 * x]) * inv_l,
+                              __uint_as_float(orr[c][2 * x + 1]) * inv_l);
+        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) d4[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  const uint32_t a = smem_addr(p);
+  return p + ((1024u - (a & 1023u)) & 1023u);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                const __grid_constant__ CUtensorMap tv, const __grid_constant__ AttnParams p) {
+  constexpr int NST = Cfg<D>::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  auto* bars = reinterpret_cast<Bars<NST>*>(smem + Cfg<D>::kBarOff);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_empty, 1);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&bars->kv_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&bars->s_full[w], 1);
+      mbar_init(&bars->p_full[w], 128);
+      mbar_init(&bars->o_full[w], 1);
+      mbar_init(&bars->o_empty[w], 128);
+    }
+    mbar_init(&bars->mma_done, 1);
+    bars->abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(&bars->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == kWarpTma && lane == 0) {
+    tma_prefetch_desc(&tq);
+    tma_prefetch_desc(&tk);
+    tma_prefetch_desc(&tv);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = bars->tmem_base;
+
+  if (warp < 8) {
+    setmaxnreg_inc<kSoftmaxRegs>();
+    softmax_role<D>(p, bars, warp >> 2, warp & 3, lane, tmem_base);
+  } else {
+    setmaxnreg_dec<kSideRegs>();
+  }
+  if (warp < 8) {
+  } else if (warp == kWarpTma) {
+    if (lane == 0) producer_role<D>(p, bars, smem, &tq, &tk, &tv);
+    __syncwarp();
+  } else if (warp == kWarpMma) {
+    if (lane == 0) mma_role<D>(p, bars, smem, tmem_base);
+    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ debug kernels
+
+__global__ void dump_tiles_kernel(Pattern pat, int nqb, int* out, long long cap) {
+  const int qb = blockIdx.x * blockDim.x + threadIdx.x;
+  if (qb >= nqb) return;
+  long long off = 0;
+  for (int q = 0; q < qb; ++q) off += block_tiles(pat, q, BM, BN).count();
+  const BlockTiles bt = block_tiles(pat, qb, BM, BN);
+  for (int t = 0; t < bt.count(); ++t) {
+    const long long rec = off + t;
+    if (rec >= cap) return;
+    const int kb = bt.kb(t);
+    out[3 * rec + 0] = qb;
+    out[3 * rec + 1] = kb;
+    out[3 * rec + 2] = tile_full(pat, qb, kb, BM, BN);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(128, 1)
+    mma_probe_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                     const __grid_constant__ CUtensorMap tv, float* s_out, float* o_out) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  constexpr int TB = Cfg<D>::kTileBytes;
+  uint64_t* bar_load = reinterpret_cast<uint64_t*>(smem + 3 * TB);
+  uint64_t* bar_mma = bar_load + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_load + 2);
+  int* abort_flag = reinterpret_cast<int*>(bar_load + 3);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(bar_load, 1);
+    mbar_init(bar_mma, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const uint32_t sq = smem_addr(smem), sk = sq + TB, sv = sq + 2 * TB;
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(bar_load, 3 * TB);
+    for (int pn = 0; pn < Cfg<D>::kPanels; ++pn) {
+      tma_load_4d(sq + pn * Cfg<D>::kPanelBytes, &tq, bar_load, pn * 64, 0, 0, 0);
+      tma_load_4d(sk + pn * Cfg<D>::kPanelBytes, &tk, bar_load, pn * 64, 0, 0, 0);
+      tma_load_4d(sv + pn * Cfg<D>::kPanelBytes, &tv, bar_load, pn * 64, 0, 0, 0);
+    }
+  }
+  bool ok = wait_bar(bar_load, 0, abort_flag, kSiteProbe);
+  if (threadIdx.x == 0 && ok) {
+    tc_fence_after();
+    issue_qk<D>(tbase, sq, sk);
+    mma_commit(bar_mma);
+  }
+  ok = ok && wait_bar(bar_mma, 0, abort_flag, kSiteProbe);
+  ok = __all_sync(0xffffffffu, ok);
+  const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+  const int r = threadIdx.x;
+  if (ok) {
+    tc_fence_after();
+    uint32_t sr[4][32];
+    for (int c = 0; c < 4; ++c) tmem_ld32(tbase + lane_addr + 32 * c, sr[c]);
+    tmem_wait_ld(sr[0]);
+    reg_fence(sr[1]);
+    reg_fence(sr[2]);
+    reg_fence(sr[3]);
+    for (int c = 0; c < 4; ++c)
+      for (int x = 0; x < 32; ++x) s_out[r * 128 + 32 * c + x] = __uint_as_float(sr[c][x]);
+    for (int h = 0; h < 2; ++h) {
+      uint32_t pk[32];
+      for (int x = 0; x < 32; ++x)
+        pk[x] = pack_bf16x2(__uint_as_float(sr[2 * h + (x >> 4)][(2 * x) & 31]),
+                            __uint_as_float(sr[2 * h + (x >> 4)][(2 * x + 1) & 31]));
+      tmem_st32(tbase + lane_addr + 32 * h, pk);
+    }
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && ok) {
+    tc_fence_after();
+    issue_pv<D>(tbase + 128, tbase, sv, 0u);
+    mma_commit(bar_mma);
+  }
+  ok = ok && wait_bar(bar_mma, 1, abort_flag, kSiteProbe);
+  ok = __all_sync(0xffffffffu, ok);
+  if (ok) {
+    tc_fence_after();
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t orr[32];
+      tmem_ld32(tbase + lane_addr + 128 + 32 * c, orr);
+      tmem_wait_ld(orr);
+      for (int x = 0; x < 32; ++x) o_out[r * D + 32 * c + x] = __uint_as_float(orr[x]);
+    }
+  }
+  if (threadIdx.x == 0) {  // nothing may still be in flight when TMEM is freed
+    mma_commit(bar_mma);
+    drain_wait(bar_mma, ok ? 0u : 1u);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 256);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct DeviceInfo {
+  bool ready = false;
+  bool supported = false;
+  int sms = 0;
+  bool attr_set[2] = {false, false};
+  bool probe_attr_set[2] = {false, false};
+};
+
+std::mutex g_mutex;
+EncodeTiledFn g_encode = nullptr;
+std::vector<DeviceInfo> g_devices;
+
+int get_encode_fn() {
+  if (g_encode) return TM_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || !fn)
+    return TM_ERR_CUDA;
+  g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  return TM_OK;
+}
+
+// Device facts, cached per device (thread-safe).
+int device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return TM_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (int rc = get_encode_fn()) return rc;
+  if (static_cast<int>(g_devices.size()) <= dev) g_devices.resize(dev + 1);
+  DeviceInfo& di = g_devices[dev];
+  if (!di.ready) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return TM_ERR_CUDA;
+    di.supported = (prop.major == 10 && prop.minor == 0);
+    di.sms = prop.multiProcessorCount;
+    di.ready = true;
+  }
+  *out = &di;
+  return di.supported ? TM_OK : TM_ERR_UNSUPPORTED;
+}
+
+// [B, N, H, D] bf16 tensor, 64-column x 128-row boxes, 128-byte swizzle.
+int encode_bnhd(CUtensorMap* m, const void* base, int B, int N, int H, int D, int box_rows) {
+  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2,
+                                 (cuuint64_t)N * H * D * 2};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? TM_OK : TM_ERR_CUDA;
+}
+
+template <int D>
+int launch_attention_d(const LaunchArgs& a, DeviceInfo* di) {
+  const int kidx = D == 128 ? 1 : 0;
+  if (!di->attr_set[kidx]) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    // setmaxnreg redistributes exactly kThreads x kLaunchRegs registers; any
+    // other launch register count could leave the increase waiting forever.
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, attn_kernel<D>) != cudaSuccess) return TM_ERR_CUDA;
+    if (fa.numRegs != kLaunchRegs) {
+      fprintf(stderr, "tm: attention kernel built with %d registers, expected %d\n", fa.numRegs,
+              kLaunchRegs);
+      return TM_ERR_UNSUPPORTED;
+    }
+    if (cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg<D>::kSmemBytes) != cudaSuccess)
+      return TM_ERR_CUDA;
+    di->attr_set[kidx] = true;
+  }
+  CUtensorMap tq, tk, tv;
+  if (encode_bnhd(&tq, a.q, a.B, a.N, a.Hq, D, BM) || encode_bnhd(&tk, a.k, a.B, a.N, a.Hkv, D, BN) ||
+      encode_bnhd(&tv, a.v, a.B, a.N, a.Hkv, D, BN))
+    return TM_ERR_CUDA;
+
+  AttnParams p;
+  p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.N = a.N;
+  p.G = a.Hq / a.Hkv;
+  p.npairs = (p.G + 1) / 2;
+  p.nqb = (a.N + BM - 1) / BM;
+  p.units = a.B * a.Hkv * p.npairs;
+  p.pat = a.pat;
+  p.sl2 = a.scale * 1.4426950408889634f;
+  p.o = static_cast<__nv_bfloat16*>(a.o);
+
+  // Persistent grid; items (longest q-blocks first) are split into contiguous
+  // runs of near-equal cost, cost = visited tiles x Q tiles of the item.
+  const long long n_items = static_cast<long long>(p.nqb) * p.units;
+  const int grid = static_cast<int>(std::min<long long>(std::min(di->sms, kMaxCtas), n_items));
+  std::vector<long long> qcost(p.nqb);
+  long long total = 0;
+  for (int qb = 0; qb < p.nqb; ++qb) {
+    qcost[qb] = block_tiles(p.pat, qb, BM, BN).count();
+    total += qcost[qb] * static_cast<long long>(a.B) * a.Hq;
+  }
+  int c = 0;
+  long long acc = 0;
+  p.cta_begin[0] = 0;
+  for (long long item = 0; item < n_items; ++item) {
+    while (c + 1 < grid &&
+           acc >= static_cast<long long>((static_cast<double>(total) * (c + 1)) / grid)) {
+      p.cta_begin[++c] = static_cast<int>(item);
+    }
+    const Item it = decode_item(p.B, p.Hkv, p.G, p.npairs, p.nqb, p.units, static_cast<int>(item));
+    acc += qcost[it.qb] * (1 + it.v1);
+  }
+  while (c + 1 <= grid) p.cta_begin[++c] = static_cast<int>(n_items);
+
+  attn_kernel<D><<<grid, kThreads, Cfg<D>::kSmemBytes, static_cast<cudaStream_t>(a.stream)>>>(
+      tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? TM_OK : TM_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_attention(const LaunchArgs& a) {
+  DeviceInfo* di = nullptr;
+  if (int rc = device_info(&di)) return rc;
+  if (a.D == 128) return launch_attention_d<128>(a, di);
+  if (a.D == 64) return launch_attention_d<64>(a, di);
+  return TM_ERR_UNSUPPORTED;
+}
+
+int launch_dump_tiles(const Pattern& pat, int* out_dev, long long cap, void* stream) {
+  const int nqb = (pat.N + BM - 1) / BM;
+  if (cap <= 0) return TM_OK;
+  dump_tiles_kernel<<<(nqb + 127) / 128, 128, 0, static_cast<cudaStream_t>(stream)>>>(pat, nqb,
+                                                                                      out_dev, cap);
+  return cudaGetLastError() == cudaSuccess ? TM_OK : TM_ERR_CUDA;
+}
+
+template <int D>
+static int launch_probe_d(const void* q, const void* k, const void* v, float* s_out, float* o_out,
+                          void* stream, DeviceInfo* di) {
+  const int kidx = D == 128 ? 1 : 0;
+  const int smem = 3 * Cfg<D>::kTileBytes + 64 + 1024;
+  if (!di->probe_attr_set[kidx]) {
+    if (cudaFuncSetAttribute(mma_probe_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return TM_ERR_CUDA;
+    di->probe_attr_set[kidx] = true;
+  }
+  CUtensorMap tq, tk, tv;
+  if (encode_bnhd(&tq, q, 1, 128, 1, D, 128) || encode_bnhd(&tk, k, 1, 128, 1, D, 128) ||
+      encode_bnhd(&tv, v, 1, 128, 1, D, 128))
+    return TM_ERR_CUDA;
+  mma_probe_kernel<D><<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, s_out,
+                                                                          o_out);
+  return cudaGetLastError() == cudaSuccess ? TM_OK : TM_ERR_CUDA;
+}
+
+int launch_mma_probe(const void* q, const void* k, const void* v, float* s_out, float* o_out,
+                     int D, void* stream) {
+  DeviceInfo* di = nullptr;
+  if (int rc = device_info(&di)) return rc;
+  if (D == 128) return launch_probe_d<128>(q, k, v, s_out, o_out, stream, di);
+  if (D == 64) return launch_probe_d<64>(q, k, v, s_out, o_out, stream, di);
+  return TM_ERR_UNSUPPORTED;
+}
+
+int read_and_clear_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return TM_ERR_CUDA;
+  int st = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&st, g_status, sizeof(int)) != cudaSuccess) return TM_ERR_CUDA;
+  if (st != kDevOk) {
+    int where = 0;
+    cudaMemcpyFromSymbol(&where, g_status_where, sizeof(int));
+    fprintf(stderr, "tm: kernel gave up on a pipeline wait (site %d)\n", where);
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return TM_ERR_CUDA;
+    return TM_ERR_TIMEOUT;
+  }
+  return TM_OK;
+}
+
+}  // namespace trimix

@@ -1,0 +1,32 @@
+// Internal interface between the C ABI (tm_api.cu) and the kernel translation
+// unit (tm_attn.cu). Not installed; not part of the public ABI.
+#pragma once
+
+#include <cstdint>
+
+#include "tm_tiles.cuh"
+
+namespace trimix {
+
+// Codes the kernels write into the device status word.
+enum DeviceStatus : int { kDevOk = 0, kDevTimeout = 1 };
+
+struct LaunchArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  int B, Hq, Hkv, N, D;
+  float scale;
+  Pattern pat;
+  void* stream;
+};
+
+// All return a tm_status value.
+int launch_attention(const LaunchArgs& a);
+int launch_dump_tiles(const Pattern& p, int* out_dev, long long cap, void* stream);
+int launch_mma_probe(const void* q, const void* k, const void* v, float* s_out, float* o_out,
+                     int D, void* stream);
+int read_and_clear_device_status(void* stream);
+
+}  // namespace trimix

@@ -1,0 +1,134 @@
+"""The C-ABI library without a GPU: it loads, exports every declared symbol,
+rejects bad arguments before touching CUDA, and its host tile-list export
+matches the oracle bit for bit."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+import long_context_prefill_trianglemix_b200 as tm
+from long_context_prefill_trianglemix_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build.build_lib()
+    yield
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "tm.h")).read()
+    return sorted(set(re.findall(r"TM_API\s+[\w\s\*]+?\b(tm_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    syms = declared_symbols()
+    assert len(syms) >= 10
+    out = subprocess.run(["nm", "-D", "--defined-only", tm.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (tm_\w+)", out))
+    for s in syms:
+        assert s in exported, s
+    assert set(tm.EXPORTED) == set(syms)
+    L = tm.lib()
+    for s in syms:
+        assert getattr(L, s) is not None
+
+
+def test_only_the_abi_is_exported():
+    out = subprocess.run(["nm", "-D", "--defined-only", tm.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    names = set(re.findall(r"\bT (\w+)", out))
+    assert {n for n in names if not n.startswith("tm_")} <= {"_init", "_fini"}
+
+
+def test_status_strings():
+    for code in (0, -1, -2, -3, -4, 99):
+        assert isinstance(tm.status_string(code), str) and tm.status_string(code)
+
+
+FAKE = 0x10000  # a 16-byte-aligned address that is never dereferenced (calls fail validation)
+
+
+@pytest.mark.parametrize("args,want", [
+    ((0, FAKE, FAKE, FAKE + 0x100000, 1, 4, 4, 64, 64, 0.1), tm.TM_ERR_INVALID_ARG),   # null q
+    ((FAKE, FAKE, FAKE, FAKE + 0x100000, 0, 4, 4, 64, 64, 0.1), tm.TM_ERR_INVALID_ARG),  # B < 1
+    ((FAKE, FAKE, FAKE, FAKE + 0x100000, 1, 4, 3, 64, 64, 0.1), tm.TM_ERR_INVALID_ARG),  # Hq % Hkv
+    ((FAKE, FAKE, FAKE, FAKE + 0x100000, 1, 4, 4, 0, 64, 0.1), tm.TM_ERR_INVALID_ARG),   # N < 1
+    ((FAKE, FAKE, FAKE, FAKE + 0x100000, 1, 4, 4, 64, 96, 0.1), tm.TM_ERR_UNSUPPORTED),  # D
+    ((FAKE + 8, FAKE, FAKE, FAKE + 0x100000, 1, 4, 4, 64, 64, 0.1), tm.TM_ERR_INVALID_ARG),  # align
+    ((FAKE, FAKE, FAKE, FAKE + 0x100, 1, 4, 4, 64, 64, 0.1), tm.TM_ERR_INVALID_ARG),     # o aliases q
+    ((FAKE, FAKE, FAKE, FAKE + 0x100000, 1, 4, 4, 64, 64, float("nan")), tm.TM_ERR_INVALID_ARG),
+])
+def test_causal_validation(args, want):
+    assert tm.lib().tm_causal_attn_fwd(*args, None) == want
+
+
+@pytest.mark.parametrize("S,W,L", [(-1, 4, 0), (0, 0, 0), (0, 4, -2)])
+def test_triangle_pattern_validation(S, W, L):
+    args = (FAKE, FAKE, FAKE, FAKE + 0x100000, 1, 4, 4, 64, 64, 0.1)
+    assert tm.lib().tm_triangle_attn_fwd(*args, S, W, L, None) == tm.TM_ERR_INVALID_ARG
+
+
+def test_layer_schedule_validation():
+    args = (FAKE, FAKE, FAKE, FAKE + 0x100000, 1, 4, 4, 64, 64, 0.1, 4, 8, 2)
+    assert tm.lib().tm_trianglemix_attn_fwd(*args, -1, 3, None) == tm.TM_ERR_INVALID_ARG
+    assert tm.lib().tm_trianglemix_attn_fwd(*args, 0, -3, None) == tm.TM_ERR_INVALID_ARG
+    # the bad window is only checked when the triangle kernel is chosen
+    bad = (FAKE, FAKE, FAKE, FAKE + 0x100000, 1, 4, 4, 64, 64, 0.1, 4, 0, 2)
+    assert tm.lib().tm_trianglemix_attn_fwd(*bad, 5, 3, None) == tm.TM_ERR_INVALID_ARG
+
+
+def test_binding_raises_on_error():
+    with pytest.raises(tm.TmError) as e:
+        tm.tm_causal_attn_fwd(0, FAKE, FAKE, FAKE + 0x100000, 1, 4, 4, 64, 64, 0.1, stream=0)
+    assert e.value.status == tm.TM_ERR_INVALID_ARG
+
+
+TILE_CASES = [(1, 0, 1, 0), (100, 3, 10, 5), (128, 16, 64, 64), (129, 16, 64, 0), (500, 0, 1, 0),
+              (512, 16, 64, 64), (1000, 64, 200, 130), (2049, 64, 300, 1), (777, 130, 129, 0),
+              (4096, 64, 1024, 128), (3000, 5000, 1, 0), (3000, 0, 5000, 0), (3000, 1, 1, 5000)]
+
+
+@pytest.mark.parametrize("N,S,W,L", TILE_CASES)
+@pytest.mark.parametrize("BM,BN", [(128, 128), (64, 128), (128, 64), (32, 32)])
+def test_host_tile_list_bit_exact(N, S, W, L, BM, BN):
+    for causal in (False, True):
+        got = tm.tm_tile_list(N, causal, S, W, L, BM, BN)
+        want = oracle.tile_list_bruteforce(N, causal, S, W, L, BM, BN)
+        np.testing.assert_array_equal(got, want)
+    np.testing.assert_array_equal(tm.tm_triangle_tile_list(N, S, W, L, BM, BN),
+                                  tm.tm_tile_list(N, False, S, W, L, BM, BN))
+
+
+@pytest.mark.parametrize("N,S,W,L", [(32768, 64, 1024, 128), (65536, 64, 1024, 128),
+                                     (131072, 64, 512, 256), (131072, 64, 2048, 256),
+                                     (131072, 64, 4096, 256), (131072, 64, 1024, 128)])
+def test_host_tile_list_bit_exact_large(N, S, W, L):
+    got = tm.tm_triangle_tile_list(N, S, W, L)
+    want = oracle.tile_list_rows(N, False, S, W, L)
+    np.testing.assert_array_equal(got, want)
+    assert tm.tm_kept_tiles(N, False, S, W, L) == len(want)
+
+
+def test_tile_list_capacity_and_count():
+    cnt = ctypes.c_longlong(0)
+    buf = np.zeros((3, 3), np.int32)
+    rc = tm.lib().tm_tile_list(512, 0, 16, 64, 64, 128, 128, buf.ctypes.data, 3, ctypes.byref(cnt))
+    assert rc == 0 and cnt.value == 10
+    np.testing.assert_array_equal(buf, tm.tm_tile_list(512, False, 16, 64, 64)[:3])
+    assert tm.lib().tm_tile_list(512, 0, 16, 64, 64, 128, 128, None, 5,
+                                 ctypes.byref(cnt)) == tm.TM_ERR_INVALID_ARG
+
+
+def test_kept_pairs_and_tiles():
+    for N, S, W, L in [(512, 16, 64, 64), (131072, 64, 2048, 256), (1000, 0, 1, 0)]:
+        assert tm.tm_triangle_kept_pairs(N, S, W, L) == oracle.kept_pairs(N, False, S, W, L)
+    assert tm.tm_kept_tiles(131072, True, 0, 1, 0) == 1024 * 1025 // 2
+    assert tm.tm_triangle_kept_pairs(10, 0, 0, 0) == -1
