@@ -118,27 +118,33 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- CPU oracle
 
-def oracle_sample(wl, W, n_rows: int, seed: int, host):
+def oracle_sample(wl, W, n_rows: int, seed: int, host, target_s: float = 0.0):
     """Time the fp64 oracle on a row sample of the triangle layer; returns
-    (seconds, tile-FLOP equivalent of the sample, cores, description)."""
+    (seconds, tile-FLOP equivalent of the sample, cores, description).
+    With target_s > 0 the sample grows (doubling the rows) until one timed
+    call lasts about target_s seconds; only that last call is reported."""
     import numpy as np
 
     import oracle
     import long_context_prefill_trianglemix_b200 as tm
     q, k, v = host
-    rng = np.random.default_rng(seed)
-    rows = sorted(rng.choice(wl.N, size=n_rows, replace=False).tolist())
     tiles = tm.tm_tile_list(wl.N, False, wl.S, W, wl.L)
     per_qb = np.bincount(tiles[:, 0], minlength=(wl.N + BM - 1) // BM)
     cores = oracle.hardware_threads()
-    t0 = time.perf_counter()
-    oracle.attention(q, k, v, wl.B, wl.Hq, wl.Hkv, wl.N, wl.D, wl.scale, False, wl.S, W, wl.L,
-                     rows=rows, nthreads=cores)
-    dt = time.perf_counter() - t0
+    while True:
+        rng = np.random.default_rng(seed)
+        rows = sorted(rng.choice(wl.N, size=min(n_rows, wl.N), replace=False).tolist())
+        t0 = time.perf_counter()
+        oracle.attention(q, k, v, wl.B, wl.Hq, wl.Hkv, wl.N, wl.D, wl.scale, False, wl.S, W,
+                         wl.L, rows=rows, nthreads=cores)
+        dt = time.perf_counter() - t0
+        if target_s <= 0 or dt >= 0.5 * target_s or n_rows >= wl.N:
+            break
+        n_rows = int(n_rows * min(64.0, max(2.0, target_s / max(dt, 1e-3))))
     # each sampled row stands for its share (1/BM) of its q-block's kept tiles
     equiv = float(sum(per_qb[r // BM] for r in rows)) * BN * 4.0 * wl.D * wl.Hq * wl.B
-    desc = (f"{n_rows} seeded random query rows x all {wl.Hq} q heads of the triangle layer "
-            f"(W={W}); credited with their share of the kept-tile FLOPs")
+    desc = (f"{len(rows)} seeded random query rows x all {wl.Hq} q heads of the triangle layer "
+            f"(W={W}), {cores} threads; credited with their share of the kept-tile FLOPs")
     return dt, equiv, cores, desc
 
 
@@ -302,7 +308,7 @@ def run_ours(args):
         "device_status": tm.status_string(status),
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        dt, equiv, cores, desc = oracle_sample(wl, W, args.cpu_rows, 7, host_np)
+        dt, equiv, cores, desc = oracle_sample(wl, W, args.cpu_rows, 7, host_np, target_s=10.0)
         line["cpu_baseline"] = {"value": equiv / dt / 1e12, "unit": UNIT, "cores": cores,
                                 "kind": "oracle", "sample": desc, "seconds": dt}
     if rank == 0:
@@ -321,8 +327,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="llama3-8b-128k", choices=sorted(I.WORKLOADS))
     ap.add_argument("--window", type=int, default=0, help="override W of the workload")
-    ap.add_argument("--cpu-rows", type=int, default=24, help="oracle rows for cpu_baseline")
-    ap.add_argument("--ref-rows", type=int, default=8, help="oracle rows per reference step")
+    ap.add_argument("--cpu-rows", type=int, default=256, help="first oracle sample for cpu_baseline")
+    ap.add_argument("--ref-rows", type=int, default=2048, help="oracle rows per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps, always

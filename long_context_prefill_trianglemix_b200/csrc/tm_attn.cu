@@ -409,8 +409,10 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
         for (int x = 0; x < 32; ++x) {
           const float a = ex2(fmaf(s[64 * h + 2 * x], sl2, neg_m));
           const float b = ex2(fmaf(s[64 * h + 2 * x + 1], sl2, neg_m));
-          rs += a + b;
           pk[x] = pack_bf16x2(a, b);
+          // l sums the same bf16-rounded weights that P.V uses, so O / l is a
+          // properly normalised average of v (a single dominant key returns v exactly)
+          rs += __uint_as_float(pk[x] << 16) + __uint_as_float(pk[x] & 0xFFFF0000u);
         }
         tmem_st32(tS + 32 * h, pk);
       }
