@@ -63,7 +63,8 @@ typedef enum {
 /*
  * Dense causal attention, keep(i, j) = j <= i. This is the "full attention"
  * the TriangleMix pages compare against (blog post, section 速度).
- * scale: the softmax scale applied to q.k (commonly 1/sqrt(D)); must be finite.
+ * scale: the softmax scale applied to q.k (commonly 1/sqrt(D)); must be finite and > 0
+ *        (masked scores are -inf before scaling).
  */
 TM_API int tm_causal_attn_fwd(const void* q, const void* k, const void* v, void* o, int B,
                               int Hq, int Hkv, int N, int D, float scale, void* stream);
@@ -137,6 +138,17 @@ TM_API int tm_debug_dump_tiles(int N, int causal, int S, int W, int L, int* out_
  */
 TM_API int tm_debug_mma_probe(const void* q, const void* k, const void* v, float* s_out,
                               float* o_out, int D, void* stream);
+
+/*
+ * Host export of the persistent work split the kernels use on a grid of
+ * num_ctas CTAs (the SM count on a B200): one record of five ints per work
+ * item, (cta, item, q-block, first q head (batch * Hq + head), number of Q
+ * tiles 1 or 2), in the order each CTA processes them. An item covers one
+ * q-block of one or two q heads that share a kv head. out: HOST buffer of
+ * 5*cap ints (NULL when cap = 0); *count receives the total. Host only.
+ */
+TM_API int tm_debug_schedule(int B, int Hq, int Hkv, int N, int causal, int S, int W, int L,
+                             int num_ctas, int* out, long long cap, long long* count);
 
 /*
  * Synchronises `stream`, then reads and clears the device status word of the

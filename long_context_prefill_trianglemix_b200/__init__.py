@@ -25,7 +25,8 @@ TM_BLOCK_M = TM_BLOCK_N = 128
 EXPORTED = (
     "tm_causal_attn_fwd", "tm_triangle_attn_fwd", "tm_trianglemix_attn_fwd",
     "tm_triangle_kept_pairs", "tm_kept_tiles", "tm_triangle_tile_list", "tm_tile_list",
-    "tm_debug_dump_tiles", "tm_debug_mma_probe", "tm_get_device_status", "tm_status_string",
+    "tm_debug_dump_tiles", "tm_debug_mma_probe", "tm_debug_schedule", "tm_get_device_status",
+    "tm_status_string",
 )
 
 
@@ -60,6 +61,8 @@ def lib() -> ctypes.CDLL:
             "tm_tile_list": (ci, [ci, ci, ci, ci, ci, ci, ci, vp, cll, ctypes.POINTER(cll)]),
             "tm_debug_dump_tiles": (ci, [ci, ci, ci, ci, ci, vp, cll, ctypes.POINTER(cll), vp]),
             "tm_debug_mma_probe": (ci, [vp, vp, vp, vp, vp, ci, vp]),
+            "tm_debug_schedule": (ci, [ci, ci, ci, ci, ci, ci, ci, ci, ci, vp, cll,
+                                       ctypes.POINTER(cll)]),
             "tm_get_device_status": (ci, [vp]),
             "tm_status_string": (ctypes.c_char_p, [ci]),
         }
@@ -155,6 +158,18 @@ def tm_debug_dump_tiles(N, causal, S, W, L, out_dev, cap, stream=None) -> int:
 def tm_debug_mma_probe(q, k, v, s_out, o_out, D, stream=None):
     return _check("tm_debug_mma_probe", lib().tm_debug_mma_probe(
         _ptr(q), _ptr(k), _ptr(v), _ptr(s_out), _ptr(o_out), D, _stream(stream)))
+
+
+def tm_debug_schedule(B, Hq, Hkv, N, causal, S, W, L, num_ctas=148) -> np.ndarray:
+    """Persistent work split as an int32 [n, 5] array: (cta, item, q-block, head0, tiles)."""
+    cnt = ctypes.c_longlong(0)
+    _check("tm_debug_schedule", lib().tm_debug_schedule(B, Hq, Hkv, N, int(causal), S, W, L,
+                                                        num_ctas, None, 0, ctypes.byref(cnt)))
+    out = np.zeros((max(cnt.value, 1), 5), np.int32)
+    _check("tm_debug_schedule", lib().tm_debug_schedule(B, Hq, Hkv, N, int(causal), S, W, L,
+                                                        num_ctas, out.ctypes.data, cnt.value,
+                                                        ctypes.byref(cnt)))
+    return out[: cnt.value]
 
 
 def tm_get_device_status(stream=None) -> int:

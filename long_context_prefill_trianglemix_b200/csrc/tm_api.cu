@@ -24,7 +24,7 @@ int validate_common(const void* q, const void* k, const void* v, void* o, int B,
   if (!q || !k || !v || !o) return TM_ERR_INVALID_ARG;
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || D < 1) return TM_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return TM_ERR_INVALID_ARG;
-  if (!std::isfinite(scale)) return TM_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return TM_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return TM_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return TM_ERR_INVALID_ARG;
   // sizes must stay inside the 32-bit indices used for rows and work items
@@ -152,6 +152,19 @@ TM_API int tm_debug_mma_probe(const void* q, const void* k, const void* v, float
   if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return TM_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return TM_ERR_UNSUPPORTED;
   return trimix::launch_mma_probe(q, k, v, s_out, o_out, D, stream);
+}
+
+TM_API int tm_debug_schedule(int B, int Hq, int Hkv, int N, int causal, int S, int W, int L,
+                             int num_ctas, int* out, long long cap, long long* count) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0 || num_ctas < 1 || cap < 0 || !count ||
+      (cap > 0 && !out))
+    return TM_ERR_INVALID_ARG;
+  if (!causal && validate_pattern(S, W, L)) return TM_ERR_INVALID_ARG;
+  if (static_cast<long long>((N + TM_BLOCK_M - 1) / TM_BLOCK_M) * B * Hkv * ((Hq / Hkv + 1) / 2) >
+      (1LL << 31) - 1)
+    return TM_ERR_INVALID_ARG;
+  return trimix::debug_schedule(B, Hq, Hkv, N, trimix::make_pattern(N, causal, S, W, L), num_ctas,
+                                out, cap, count);
 }
 
 TM_API int tm_get_device_status(void* stream) { return trimix::read_and_clear_device_status(stream); }

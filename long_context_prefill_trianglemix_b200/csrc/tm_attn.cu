@@ -10,7 +10,7 @@
 //   warps 0-3  softmax warpgroup 0: rows of Q tile 0 (TMEM lanes 0..127)
 //   warps 4-7  softmax warpgroup 1: rows of Q tile 1
 //   warp  8    TMA producer (one elected thread): Q tiles, then K/V tiles
-//   warp  9    tcgen05 issuer (one elected thread) and TMEM owner
+//   warp  9    tcgen05 issuer (one thread) and TMEM owner
 //   warps 10-11 idle (they complete the third warpgroup for setmaxnreg)
 // The kernel is launched at 168 registers per thread (384 x 168 = 64512);
 // the third warpgroup drops to 88 and the softmax warpgroups rise to 208
@@ -71,6 +71,16 @@ constexpr uint32_t kTmemCols = 512;
 // in fp32/bf16, and the O rescale (a TMEM round trip) becomes rare.
 constexpr float kRescaleThreshold = 8.0f;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+#ifndef TM_POLY_PAIRS
+#define TM_POLY_PAIRS 0
+#endif
+// Of every 32 pairs of probabilities, this many are exponentiated on the FMA
+// pipe (ex2_poly) and the rest on MUFU, to balance the two units.
+constexpr int kPolyPairs = TM_POLY_PAIRS;
+static_assert(kPolyPairs >= 0 && kPolyPairs <= 32, "pairs per 32");
+// Per-item fixed cost (Q load, first S, last P.V, epilogue) in units of one
+// visited tile, used only to balance the persistent work split.
+constexpr long long kItemOverheadTiles = 3;
 constexpr uint64_t kDrainLimitNs = 100000000ull;
 
 // Where a wait gave up (recorded with the timeout, for diagnosis).
@@ -109,8 +119,30 @@ struct AttnParams {
   Pattern pat;
   float sl2;  // softmax scale * log2(e)
   __nv_bfloat16* o;
-  int cta_begin[kMaxCtas + 1];
+  // Work of CTA c: the big items c, c + grid, c + 2 grid, ... below n_big (dealt
+  // round-robin, longest first), then the contiguous run [run_begin[c],
+  // run_begin[c + 1]) of the remaining items.
+  int n_big;
+  int run_begin[kMaxCtas + 1];
 };
+
+__host__ __device__ __forceinline__ int work_count(const AttnParams& p, int c, int g) {
+  const int nb = c < p.n_big ? (p.n_big - c + g - 1) / g : 0;
+  return nb + p.run_begin[c + 1] - p.run_begin[c];
+}
+
+__host__ __device__ __forceinline__ int work_item(const AttnParams& p, int c, int g, int k) {
+  const int nb = c < p.n_big ? (p.n_big - c + g - 1) / g : 0;
+  return k < nb ? c + k * g : p.run_begin[c] + (k - nb);
+}
+
+__device__ __forceinline__ int cta_work_count(const AttnParams& p) {
+  return work_count(p, blockIdx.x, gridDim.x);
+}
+
+__device__ __forceinline__ int cta_work_item(const AttnParams& p, int k) {
+  return work_item(p, blockIdx.x, gridDim.x, k);
+}
 
 struct Item {
   int b, g, qb, h0, v1;
@@ -167,25 +199,28 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 // ------------------------------------------------------------------ MMA helpers
 
 // S[128 x 128] = Q[128 x D] . K[128 x D]^T; both tiles K-major, 128B-swizzled,
-// stored as D/64 panels of 128 rows x 128 bytes.
+// stored as D/64 panels of 128 rows x 128 bytes. q_lo / k_lo: low descriptor
+// words of the tiles (desc_lo_sw128 with LBO 16); a k-step of 16 columns is
+// +32 bytes inside a panel, the next panel +kPanelBytes.
 template <int D>
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_base, uint32_t k_base) {
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_lo, uint32_t k_lo) {
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk >> 2) * Cfg<D>::kPanelBytes + (kk & 3) * 32;
-    mma_ss(d_tmem, smem_desc_sw128(q_base + off, 16, 1024), smem_desc_sw128(k_base + off, 16, 1024),
+    const uint32_t off = ((kk >> 2) * Cfg<D>::kPanelBytes + (kk & 3) * 32) >> 4;
+    mma_ss(d_tmem, desc_join(q_lo + off, kDescHiSw128), desc_join(k_lo + off, kDescHiSw128),
            Cfg<D>::kIdescS, kk > 0 ? 1u : 0u);
   }
 }
 
 // O[128 x D] (+)= P[128 x 128] (bf16 in TMEM, 2 per column) . V[128 x D];
-// V is MN-major (D contiguous per key row): 16 keys per step = 16 rows.
+// V is MN-major (D contiguous per key row): 16 keys per step = 16 rows = 2048
+// bytes. v_lo: low descriptor word of the V tile (LBO = one panel).
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_base,
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_lo,
                                          uint32_t accumulate) {
 #pragma unroll
   for (int kk = 0; kk < BN / 16; ++kk) {
-    mma_ts(d_tmem, p_tmem + kk * 8, smem_desc_sw128(v_base + kk * 16 * 128, Cfg<D>::kPanelBytes, 1024),
+    mma_ts(d_tmem, p_tmem + kk * 8, desc_join(v_lo + kk * (2048 >> 4), kDescHiSw128),
            Cfg<D>::kIdescO, (accumulate || kk > 0) ? 1u : 0u);
   }
 }
@@ -218,8 +253,9 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, Bars<Cfg<D>::
   const uint32_t ring = smem_addr(smem + Cfg<D>::kRingOff);
   uint32_t kv_cnt = 0, it_cnt = 0;
   bool ok = true;
-  for (int item = p.cta_begin[blockIdx.x]; ok && item < p.cta_begin[blockIdx.x + 1]; ++item) {
-    const Item it = decode_item(p.B, p.Hkv, p.G, p.npairs, p.nqb, p.units, item);
+  const int n_work = cta_work_count(p);
+  for (int k = 0; ok && k < n_work; ++k) {
+    const Item it = decode_item(p.B, p.Hkv, p.G, p.npairs, p.nqb, p.units, cta_work_item(p, k));
     const BlockTiles bt = block_tiles(p.pat, it.qb, BM, BN);
     if (!(ok = wait_bar(&bars->q_empty, (it_cnt & 1u) ^ 1u, abort_flag, kSiteQEmpty))) break;
     mbar_arrive_expect_tx(&bars->q_full, (1 + it.v1) * Cfg<D>::kTileBytes);
@@ -257,13 +293,21 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, Bars<Cfg<D>::
   }
 }
 
+// The tcgen05 issuer: one thread issues every MMA of both Q tiles in the order
+// O0+=P0.V_t, S0=Q0.K_{t+1}, O1+=P1.V_t, S1=Q1.K_{t+1}. Descriptors are kept as
+// precomputed low words plus per-k-step constant adds: the issuing warp shares
+// its SM sub-partition with two softmax warps, so every instruction it saves
+// per MMA shortens the time the tensor pipe waits for the next one.
 template <int D>
 __device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStages>* bars,
                                          uint8_t* smem, uint32_t tmem_base) {
   constexpr int NST = Cfg<D>::kStages;
   volatile int* abort_flag = &bars->abort_flag;
-  const uint32_t q0 = smem_addr(smem), q1 = q0 + Cfg<D>::kTileBytes;
+  const uint32_t q0 = desc_lo_sw128(smem_addr(smem), 16), q1 = desc_lo_sw128(smem_addr(smem) + Cfg<D>::kTileBytes, 16);
   const uint32_t ring = smem_addr(smem + Cfg<D>::kRingOff);
+  const uint32_t k_lo0 = desc_lo_sw128(ring, 16);
+  const uint32_t v_lo0 = desc_lo_sw128(ring, Cfg<D>::kPanelBytes);
+  constexpr uint32_t kStageLo = Cfg<D>::kTileBytes >> 4;
   const uint32_t tS0 = tmem_base + Cfg<D>::kTmemS0, tS1 = tmem_base + Cfg<D>::kTmemS1;
   const uint32_t tO0 = tmem_base + Cfg<D>::kTmemO0, tO1 = tmem_base + Cfg<D>::kTmemO1;
   uint32_t kv_cnt = 0, it_cnt = 0, pc0 = 0, pc1 = 0, oe0 = 0, oe1 = 0;
@@ -271,18 +315,19 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStag
 #define TM_WAIT(bar, par, site)                                      \
   if (!(ok = wait_bar((bar), (par), abort_flag, (site)))) break; \
   tc_fence_after();
-  for (int item = p.cta_begin[blockIdx.x]; ok && item < p.cta_begin[blockIdx.x + 1]; ++item) {
-    const Item it = decode_item(p.B, p.Hkv, p.G, p.npairs, p.nqb, p.units, item);
+  const int n_work = cta_work_count(p);
+  for (int k = 0; ok && k < n_work; ++k) {
+    const Item it = decode_item(p.B, p.Hkv, p.G, p.npairs, p.nqb, p.units, cta_work_item(p, k));
     const int T = block_tiles(p.pat, it.qb, BM, BN).count();
     const bool v1 = it.v1 != 0;
     TM_WAIT(&bars->q_full, it_cnt & 1u, kSiteQFull);
     ++it_cnt;
     uint32_t kst = kv_cnt % NST;
     TM_WAIT(&bars->kv_full[kst], (kv_cnt / NST) & 1u, kSiteKvFull);
-    issue_qk<D>(tS0, q0, ring + kst * Cfg<D>::kTileBytes);
+    issue_qk<D>(tS0, q0, k_lo0 + kst * kStageLo);
     mma_commit(&bars->s_full[0]);
     if (v1) {
-      issue_qk<D>(tS1, q1, ring + kst * Cfg<D>::kTileBytes);
+      issue_qk<D>(tS1, q1, k_lo0 + kst * kStageLo);
       mma_commit(&bars->s_full[1]);
     }
     if (T == 1) mma_commit(&bars->q_empty);
@@ -297,13 +342,13 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStag
       }
       TM_WAIT(&bars->p_full[0], pc0 & 1u, kSitePFull);
       ++pc0;
-      issue_pv<D>(tO0, tS0, ring + vst * Cfg<D>::kTileBytes, t > 0 ? 1u : 0u);
+      issue_pv<D>(tO0, tS0, v_lo0 + vst * kStageLo, t > 0 ? 1u : 0u);
       if (t == T - 1) mma_commit(&bars->o_full[0]);
       if (t + 1 < T) {
         const uint32_t kidx = kv_cnt + 1;
         kst = kidx % NST;
         TM_WAIT(&bars->kv_full[kst], (kidx / NST) & 1u, kSiteKvFull);
-        issue_qk<D>(tS0, q0, ring + kst * Cfg<D>::kTileBytes);
+        issue_qk<D>(tS0, q0, k_lo0 + kst * kStageLo);
         mma_commit(&bars->s_full[0]);
         if (!v1 && t + 1 == T - 1) mma_commit(&bars->q_empty);
       }
@@ -314,14 +359,14 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStag
         }
         TM_WAIT(&bars->p_full[1], pc1 & 1u, kSitePFull);
         ++pc1;
-        issue_pv<D>(tO1, tS1, ring + vst * Cfg<D>::kTileBytes, t > 0 ? 1u : 0u);
+        issue_pv<D>(tO1, tS1, v_lo0 + vst * kStageLo, t > 0 ? 1u : 0u);
         if (t == T - 1) mma_commit(&bars->o_full[1]);
       }
       mma_commit(&bars->kv_empty[vst]);  // V_t free once both P.V products are done
       ++kv_cnt;
       if (t + 1 < T) {
         if (v1) {
-          issue_qk<D>(tS1, q1, ring + kst * Cfg<D>::kTileBytes);
+          issue_qk<D>(tS1, q1, k_lo0 + kst * kStageLo);
           mma_commit(&bars->s_full[1]);
           if (t + 1 == T - 1) mma_commit(&bars->q_empty);
         }
@@ -347,8 +392,9 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
   const float sl2 = p.sl2;
   const Pattern& pat = p.pat;
   uint32_t s_cnt = 0, o_cnt = 0;
-  for (int item = p.cta_begin[blockIdx.x]; item < p.cta_begin[blockIdx.x + 1]; ++item) {
-    const Item it = decode_item(p.B, p.Hkv, p.G, p.npairs, p.nqb, p.units, item);
+  const int n_work = cta_work_count(p);
+  for (int k = 0; k < n_work; ++k) {
+    const Item it = decode_item(p.B, p.Hkv, p.G, p.npairs, p.nqb, p.units, cta_work_item(p, k));
     if (wg == 1 && !it.v1) continue;
     const BlockTiles bt = block_tiles(pat, it.qb, BM, BN);
     const int T = bt.count();
@@ -390,9 +436,16 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
       for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int x = 0; x < 32; ++x) s[32 * c + x] = __uint_as_float(sr[c][x]);
-      float mx = s[0];
+      // row max: 3-input max over eight independent chains
+      float mxa[8];
 #pragma unroll
-      for (int x = 1; x < 128; ++x) mx = fmaxf(mx, s[x]);
+      for (int y = 0; y < 8; ++y) mxa[y] = fmaxf(s[2 * y], s[2 * y + 1]);
+#pragma unroll
+      for (int x = 16; x < 128; x += 16)
+#pragma unroll
+        for (int y = 0; y < 8; ++y) mxa[y] = fmax3(mxa[y], s[x + 2 * y], s[x + 2 * y + 1]);
+      const float mx = fmaxf(fmax3(mxa[0], mxa[1], mxa[2]),
+                             fmax3(fmax3(mxa[3], mxa[4], mxa[5]), mxa[6], mxa[7]));
       const float m_new = fmaxf(m_run, mx * sl2);
       const bool bump = m_new > m_run + kRescaleThreshold;
       float alpha = 1.f;
@@ -401,21 +454,26 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
         m_run = m_new;
       }
       const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
-      float rs = 0.f;
+      // p = 2^(s * scale * log2 e - m): packed fp32x2 FMA, then exp2; l sums the
+      // same bf16-rounded weights that P.V uses (exact widening adds), so O / l is
+      // a properly normalised average of v (a single dominant key returns v exactly)
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t pk[32];
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
-          const float a = ex2(fmaf(s[64 * h + 2 * x], sl2, neg_m));
-          const float b = ex2(fmaf(s[64 * h + 2 * x + 1], sl2, neg_m));
+          // the first kPolyPairs pairs of every 32 use the FMA-pipe exp2, the rest MUFU
+          float xa, xb;
+          ffma2(xa, xb, s[64 * h + 2 * x], s[64 * h + 2 * x + 1], sl2, sl2, neg_m, neg_m);
+          const float a = x < kPolyPairs ? ex2_poly(xa) : ex2(xa);
+          const float b = x < kPolyPairs ? ex2_poly(xb) : ex2(xb);
           pk[x] = pack_bf16x2(a, b);
-          // l sums the same bf16-rounded weights that P.V uses, so O / l is a
-          // properly normalised average of v (a single dominant key returns v exactly)
-          rs += __uint_as_float(pk[x] << 16) + __uint_as_float(pk[x] & 0xFFFF0000u);
+          add_bf16x2_to_f32(acc[2 * (x & 3)], acc[2 * (x & 3) + 1], pk[x]);
         }
         tmem_st32(tS + 32 * h, pk);
       }
+      const float rs = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
       l_run = l_run * alpha + rs;
       if (t > 0 && __any_sync(0xffffffffu, bump)) {
 #pragma unroll
@@ -590,7 +648,7 @@ __global__ void __launch_bounds__(128, 1)
   bool ok = wait_bar(bar_load, 0, abort_flag, kSiteProbe);
   if (threadIdx.x == 0 && ok) {
     tc_fence_after();
-    issue_qk<D>(tbase, sq, sk);
+    issue_qk<D>(tbase, desc_lo_sw128(sq, 16), desc_lo_sw128(sk, 16));
     mma_commit(bar_mma);
   }
   ok = ok && wait_bar(bar_mma, 0, abort_flag, kSiteProbe);
@@ -620,7 +678,7 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   if (threadIdx.x == 0 && ok) {
     tc_fence_after();
-    issue_pv<D>(tbase + 128, tbase, sv, 0u);
+    issue_pv<D>(tbase + 128, tbase, desc_lo_sw128(sv, Cfg<D>::kPanelBytes), 0u);
     mma_commit(bar_mma);
   }
   ok = ok && wait_bar(bar_mma, 1, abort_flag, kSiteProbe);
@@ -711,6 +769,64 @@ int encode_bnhd(CUtensorMap* m, const void* base, int B, int N, int H, int D, in
   return r == CUDA_SUCCESS ? TM_OK : TM_ERR_CUDA;
 }
 
+// Fills the geometry and the persistent work split of *p; returns the grid size.
+int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ctas, AttnParams* p) {
+  p->B = B; p->Hq = Hq; p->Hkv = Hkv; p->N = N;
+  p->G = Hq / Hkv;
+  p->npairs = (p->G + 1) / 2;
+  p->nqb = (N + BM - 1) / BM;
+  p->units = B * Hkv * p->npairs;
+  p->pat = pat;
+  // Persistent grid. Item cost = (visited tiles + fixed per-item overhead,
+  // about the pipeline fill/drain and epilogue) x Q tiles of the item. Items
+  // costing more than a quarter of a CTA's share (the last-L q-blocks of the
+  // triangle) are dealt round-robin first, longest first; the rest are split
+  // into contiguous runs sized by what each CTA still has room for.
+  const long long n_items = static_cast<long long>(p->nqb) * p->units;
+  const int grid = static_cast<int>(std::min<long long>(std::min(max_ctas, kMaxCtas), n_items));
+  std::vector<long long> qcost(p->nqb);
+  long long total = 0;
+  for (int qb = 0; qb < p->nqb; ++qb) {
+    qcost[qb] = block_tiles(p->pat, qb, BM, BN).count() + kItemOverheadTiles;
+    total += qcost[qb] * static_cast<long long>(B) * Hq;
+  }
+  auto item_cost = [&](long long item) {
+    const Item it = decode_item(p->B, p->Hkv, p->G, p->npairs, p->nqb, p->units, static_cast<int>(item));
+    return qcost[it.qb] * (1 + it.v1);
+  };
+  const double target = static_cast<double>(total) / grid;
+  long long n_big = 0;
+  while (n_big < n_items && n_big < 8LL * grid && 4.0 * item_cost(n_big) > target) ++n_big;
+  std::vector<double> cap(grid, target);
+  double big_total = 0;
+  for (long long j = 0; j < n_big; ++j) {
+    const double c = static_cast<double>(item_cost(j));
+    cap[j % grid] -= c;
+    big_total += c;
+  }
+  double cap_total = 0;
+  for (int c = 0; c < grid; ++c) cap_total += std::max(0.0, cap[c]);
+  const double rest = static_cast<double>(total) - big_total;
+  p->n_big = static_cast<int>(n_big);
+  p->run_begin[0] = static_cast<int>(n_big);
+  int c = 0;
+  double acc = 0, bound = 0;
+  auto next_bound = [&](int cc) {
+    return cap_total > 0 ? bound + rest * std::max(0.0, cap[cc]) / cap_total : rest * (cc + 1) / grid;
+  };
+  bound = next_bound(0);
+  for (long long item = n_big; item < n_items; ++item) {
+    while (c + 1 < grid && acc >= bound) {
+      p->run_begin[++c] = static_cast<int>(item);
+      bound = next_bound(c);
+    }
+    acc += static_cast<double>(item_cost(item));
+  }
+  while (c + 1 <= grid) p->run_begin[++c] = static_cast<int>(n_items);
+
+  return grid;
+}
+
 template <int D>
 int launch_attention_d(const LaunchArgs& a, DeviceInfo* di) {
   const int kidx = D == 128 ? 1 : 0;
@@ -736,38 +852,10 @@ int launch_attention_d(const LaunchArgs& a, DeviceInfo* di) {
     return TM_ERR_CUDA;
 
   AttnParams p;
-  p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.N = a.N;
-  p.G = a.Hq / a.Hkv;
-  p.npairs = (p.G + 1) / 2;
-  p.nqb = (a.N + BM - 1) / BM;
-  p.units = a.B * a.Hkv * p.npairs;
-  p.pat = a.pat;
   p.sl2 = a.scale * 1.4426950408889634f;
   p.o = static_cast<__nv_bfloat16*>(a.o);
 
-  // Persistent grid; items (longest q-blocks first) are split into contiguous
-  // runs of near-equal cost, cost = visited tiles x Q tiles of the item.
-  const long long n_items = static_cast<long long>(p.nqb) * p.units;
-  const int grid = static_cast<int>(std::min<long long>(std::min(di->sms, kMaxCtas), n_items));
-  std::vector<long long> qcost(p.nqb);
-  long long total = 0;
-  for (int qb = 0; qb < p.nqb; ++qb) {
-    qcost[qb] = block_tiles(p.pat, qb, BM, BN).count();
-    total += qcost[qb] * static_cast<long long>(a.B) * a.Hq;
-  }
-  int c = 0;
-  long long acc = 0;
-  p.cta_begin[0] = 0;
-  for (long long item = 0; item < n_items; ++item) {
-    while (c + 1 < grid &&
-           acc >= static_cast<long long>((static_cast<double>(total) * (c + 1)) / grid)) {
-      p.cta_begin[++c] = static_cast<int>(item);
-    }
-    const Item it = decode_item(p.B, p.Hkv, p.G, p.npairs, p.nqb, p.units, static_cast<int>(item));
-    acc += qcost[it.qb] * (1 + it.v1);
-  }
-  while (c + 1 <= grid) p.cta_begin[++c] = static_cast<int>(n_items);
-
+  const int grid = build_schedule(a.B, a.Hq, a.Hkv, a.N, a.pat, di->sms, &p);
   attn_kernel<D><<<grid, kThreads, Cfg<D>::kSmemBytes, static_cast<cudaStream_t>(a.stream)>>>(
       tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? TM_OK : TM_ERR_CUDA;
@@ -781,6 +869,25 @@ int launch_attention(const LaunchArgs& a) {
   if (a.D == 128) return launch_attention_d<128>(a, di);
   if (a.D == 64) return launch_attention_d<64>(a, di);
   return TM_ERR_UNSUPPORTED;
+}
+
+int debug_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ctas, int* out,
+                   long long cap, long long* count) {
+  AttnParams p;
+  const int grid = build_schedule(B, Hq, Hkv, N, pat, max_ctas, &p);
+  long long n = 0;
+  for (int c = 0; c < grid; ++c) {
+    const int nw = work_count(p, c, grid);
+    for (int k = 0; k < nw; ++k, ++n) {
+      if (n >= cap) continue;
+      const int item = work_item(p, c, grid, k);
+      const Item it = decode_item(p.B, p.Hkv, p.G, p.npairs, p.nqb, p.units, item);
+      int* r = out + 5 * n;
+      r[0] = c; r[1] = item; r[2] = it.qb; r[3] = it.b * Hq + it.h0; r[4] = 1 + it.v1;
+    }
+  }
+  *count = n;
+  return TM_OK;
 }
 
 int launch_dump_tiles(const Pattern& pat, int* out_dev, long long cap, void* stream) {

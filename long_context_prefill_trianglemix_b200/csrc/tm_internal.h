@@ -28,5 +28,7 @@ int launch_dump_tiles(const Pattern& p, int* out_dev, long long cap, void* strea
 int launch_mma_probe(const void* q, const void* k, const void* v, float* s_out, float* o_out,
                      int D, void* stream);
 int read_and_clear_device_status(void* stream);
+int debug_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ctas, int* out,
+                   long long cap, long long* count);
 
 }  // namespace trimix

@@ -5,6 +5,8 @@
 
 #include <cstdint>
 
+#include "tm_exp2_poly.h"
+
 namespace trimix {
 namespace sm100 {
 
@@ -192,6 +194,21 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// The same descriptor as two 32-bit words, so that per-k-step offsets are one
+// 32-bit add on the low word (the 14-bit address field never carries: shared
+// addresses stay below 256 KB). desc_lo_sw128 holds the address and LBO,
+// kDescHiSw128 the SBO of 1024 bytes, version 1 and SWIZZLE_128B.
+__host__ __device__ constexpr uint32_t desc_lo_sw128(uint32_t saddr, uint32_t lbo_bytes) {
+  return ((saddr & 0x3FFFFu) >> 4) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+constexpr uint32_t kDescHiSw128 = ((1024u >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+
+__device__ __forceinline__ uint64_t desc_join(uint32_t lo, uint32_t hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
+  return d;
+}
+
 // Instruction descriptor, kind::f16 with bf16 A and B, fp32 D.
 // a_mn_major / b_mn_major: 0 = K-major, 1 = MN-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_major,
@@ -223,6 +240,45 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA and integer pipes instead of MUFU: x = n + f with n = round(x)
+// (adding 1.5 * 2^23 rounds x to an integer inside the FADD), 2^f from the
+// fitted cubic in tm_exp2_poly.h (relative error below 1e-4, far under bf16's
+// 2^-9), and 2^n applied by adding n to the exponent field. x is clamped at
+// -125 so the exponent stays normal: -inf yields about 2^-125 instead of 0,
+// which is negligible next to a row's largest weight (at least 1).
+__device__ __forceinline__ float ex2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  const float p = fmaf(fmaf(fmaf(TM_EXP2_C3, f, TM_EXP2_C2), f, TM_EXP2_C1), f, TM_EXP2_C0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// (d0, d1) = (a0, a1) * (b0, b1) + (c0, c1) as one packed fp32x2 FMA.
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
+                                      float c0, float c1) {
+  asm("{\n\t.reg .b64 a, b, c, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+// max of three floats in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// acc_lo += bf16 low half of w, acc_hi += bf16 high half of w (exact widening adds).
+__device__ __forceinline__ void add_bf16x2_to_f32(float& acc_lo, float& acc_hi, uint32_t w) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "add.rn.f32.bf16 %0, l, %0;\n\tadd.rn.f32.bf16 %1, h, %1;\n\t}"
+      : "+f"(acc_lo), "+f"(acc_hi)
+      : "r"(w));
 }
 
 // Two floats -> packed bf16x2 (round to nearest even); `lo` lands in bits 0..15.

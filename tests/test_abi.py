@@ -65,6 +65,8 @@ FAKE = 0x10000  # a 16-byte-aligned address that is never dereferenced (calls fa
     ((FAKE + 8, FAKE, FAKE, FAKE + 0x100000, 1, 4, 4, 64, 64, 0.1), tm.TM_ERR_INVALID_ARG),  # align
     ((FAKE, FAKE, FAKE, FAKE + 0x100, 1, 4, 4, 64, 64, 0.1), tm.TM_ERR_INVALID_ARG),     # o aliases q
     ((FAKE, FAKE, FAKE, FAKE + 0x100000, 1, 4, 4, 64, 64, float("nan")), tm.TM_ERR_INVALID_ARG),
+    ((FAKE, FAKE, FAKE, FAKE + 0x100000, 1, 4, 4, 64, 64, 0.0), tm.TM_ERR_INVALID_ARG),
+    ((FAKE, FAKE, FAKE, FAKE + 0x100000, 1, 4, 4, 64, 64, -0.5), tm.TM_ERR_INVALID_ARG),
 ])
 def test_causal_validation(args, want):
     assert tm.lib().tm_causal_attn_fwd(*args, None) == want
