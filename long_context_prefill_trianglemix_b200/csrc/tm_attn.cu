@@ -22,6 +22,9 @@
 // masking runs only on the tiles that need it.
 //
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).
+// The output leaves through shared memory and TMA stores (one 4 KB slot per
+// softmax warp), so the epilogue does not flood the load/store path with
+// scattered 16-byte global writes while the other warpgroup is still working.
 // P (bf16) overwrites the first 64 columns of its S tile once S has been read
 // into registers, and feeds the P.V MMA directly from TMEM.
 //
@@ -96,7 +99,11 @@ struct Cfg {
   static constexpr int kPanels = D / 64;
   static constexpr int kStages = (D == 128) ? 4 : 8;
   static constexpr int kRingOff = 2 * kTileBytes;
-  static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
+  // Output staging: one 4 KB slot per softmax warp (32 rows x 64 bf16 columns,
+  // 128-byte swizzled), written from registers and sent out by a TMA store.
+  static constexpr int kStageOff = kRingOff + kStages * kTileBytes;
+  static constexpr int kStageSlotBytes = 32 * 128;
+  static constexpr int kBarOff = kStageOff + 8 * kStageSlotBytes;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // barriers + alignment slack
   static constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128;
   static constexpr uint32_t kTmemO0 = 256, kTmemO1 = 256 + D;
@@ -118,7 +125,6 @@ struct AttnParams {
   int B, Hq, Hkv, N, G, npairs, nqb, units;
   Pattern pat;
   float sl2;  // softmax scale * log2(e)
-  __nv_bfloat16* o;
   // Work of CTA c: the big items c, c + grid, c + 2 grid, ... below n_big (dealt
   // round-robin, longest first), then the contiguous run [run_begin[c],
   // run_begin[c + 1]) of the remaining items.
@@ -134,14 +140,6 @@ __host__ __device__ __forceinline__ int work_count(const AttnParams& p, int c, i
 __host__ __device__ __forceinline__ int work_item(const AttnParams& p, int c, int g, int k) {
   const int nb = c < p.n_big ? (p.n_big - c + g - 1) / g : 0;
   return k < nb ? c + k * g : p.run_begin[c] + (k - nb);
-}
-
-__device__ __forceinline__ int cta_work_count(const AttnParams& p) {
-  return work_count(p, blockIdx.x, gridDim.x);
-}
-
-__device__ __forceinline__ int cta_work_item(const AttnParams& p, int k) {
-  return work_item(p, blockIdx.x, gridDim.x, k);
 }
 
 struct Item {
@@ -163,6 +161,57 @@ __host__ __device__ __forceinline__ Item decode_item(int B, int Hkv, int G, int 
   it.v1 = (2 * pr + 1 < G) ? 1 : 0;
   return it;
 }
+
+// Walks one CTA's work (the same sequence as work_item) without integer
+// division per item: an integer division costs a MUFU reciprocal, and MUFU is
+// the unit the softmax warps keep busy with exp2. Big items are decoded
+// directly (a few per CTA); the contiguous run advances pair -> kv head ->
+// batch -> q-block with carries.
+struct WorkCursor {
+  int k, n_work, nb, big_next, g;
+  int qi, pr, kvh, b;  // position of the next run item
+  __host__ __device__ __forceinline__ void init(const AttnParams& p, int c, int grid) {
+    g = grid;
+    nb = c < p.n_big ? (p.n_big - c + g - 1) / g : 0;
+    n_work = nb + p.run_begin[c + 1] - p.run_begin[c];
+    k = 0;
+    big_next = c;
+    const int item = p.run_begin[c];
+    qi = item / p.units;
+    const int u = item - qi * p.units;
+    pr = u % p.npairs;
+    const int gb = u / p.npairs;
+    kvh = gb % p.Hkv;
+    b = gb / p.Hkv;
+  }
+  __host__ __device__ __forceinline__ bool done() const { return k >= n_work; }
+  // Returns the next item of this CTA and advances.
+  __host__ __device__ __forceinline__ Item next(const AttnParams& p) {
+    Item it;
+    if (k < nb) {
+      it = decode_item(p.B, p.Hkv, p.G, p.npairs, p.nqb, p.units, big_next);
+      big_next += g;
+    } else {
+      it.qb = p.nqb - 1 - qi;
+      it.g = kvh;
+      it.b = b;
+      it.h0 = kvh * p.G + 2 * pr;
+      it.v1 = (2 * pr + 1 < p.G) ? 1 : 0;
+      if (++pr == p.npairs) {
+        pr = 0;
+        if (++kvh == p.Hkv) {
+          kvh = 0;
+          if (++b == p.B) {
+            b = 0;
+            ++qi;
+          }
+        }
+      }
+    }
+    ++k;
+    return it;
+  }
+};
 
 __device__ __forceinline__ void record_timeout(int site) {
   if (atomicCAS(&g_status, kDevOk, kDevTimeout) == kDevOk) g_status_where = site;
@@ -253,9 +302,10 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, Bars<Cfg<D>::
   const uint32_t ring = smem_addr(smem + Cfg<D>::kRingOff);
   uint32_t kv_cnt = 0, it_cnt = 0;
   bool ok = true;
-  const int n_work = cta_work_count(p);
-  for (int k = 0; ok && k < n_work; ++k) {
-    const Item it = decode_item(p.B, p.Hkv, p.G, p.npairs, p.nqb, p.units, cta_work_item(p, k));
+  WorkCursor cur;
+  cur.init(p, blockIdx.x, gridDim.x);
+  while (ok && !cur.done()) {
+    const Item it = cur.next(p);
     const BlockTiles bt = block_tiles(p.pat, it.qb, BM, BN);
     if (!(ok = wait_bar(&bars->q_empty, (it_cnt & 1u) ^ 1u, abort_flag, kSiteQEmpty))) break;
     mbar_arrive_expect_tx(&bars->q_full, (1 + it.v1) * Cfg<D>::kTileBytes);
@@ -315,9 +365,10 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStag
 #define TM_WAIT(bar, par, site)                                      \
   if (!(ok = wait_bar((bar), (par), abort_flag, (site)))) break; \
   tc_fence_after();
-  const int n_work = cta_work_count(p);
-  for (int k = 0; ok && k < n_work; ++k) {
-    const Item it = decode_item(p.B, p.Hkv, p.G, p.npairs, p.nqb, p.units, cta_work_item(p, k));
+  WorkCursor cur;
+  cur.init(p, blockIdx.x, gridDim.x);
+  while (ok && !cur.done()) {
+    const Item it = cur.next(p);
     const int T = block_tiles(p.pat, it.qb, BM, BN).count();
     const bool v1 = it.v1 != 0;
     TM_WAIT(&bars->q_full, it_cnt & 1u, kSiteQFull);
@@ -383,7 +434,8 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStag
 
 template <int D>
 __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::kStages>* bars,
-                                             int wg, int wq, int lane, uint32_t tmem_base) {
+                                             uint8_t* smem, const CUtensorMap* to, int wg, int wq,
+                                             int lane, uint32_t tmem_base) {
   volatile int* abort_flag = &bars->abort_flag;
   const int r = wq * 32 + lane;  // row of the Q tile == TMEM lane
   const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
@@ -392,9 +444,10 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
   const float sl2 = p.sl2;
   const Pattern& pat = p.pat;
   uint32_t s_cnt = 0, o_cnt = 0;
-  const int n_work = cta_work_count(p);
-  for (int k = 0; k < n_work; ++k) {
-    const Item it = decode_item(p.B, p.Hkv, p.G, p.npairs, p.nqb, p.units, cta_work_item(p, k));
+  WorkCursor cur;
+  cur.init(p, blockIdx.x, gridDim.x);
+  while (!cur.done()) {
+    const Item it = cur.next(p);
     if (wg == 1 && !it.v1) continue;
     const BlockTiles bt = block_tiles(pat, it.qb, BM, BN);
     const int T = bt.count();
@@ -490,7 +543,8 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
       tc_fence_before();
       mbar_arrive(&bars->p_full[wg]);
     }
-    // epilogue: O / l -> bf16 -> global
+    // epilogue: O / l -> bf16 -> this warp's 128B-swizzled staging slot (32 rows x
+    // 64 columns at a time) -> one TMA store per half; rows past N are clipped.
     bool ok = wait_bar(&bars->o_full[wg], o_cnt & 1u, abort_flag, kSiteOFull);
     ++o_cnt;
     if (!__all_sync(0xffffffffu, ok)) return;
@@ -504,19 +558,26 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
     tc_fence_before();
     mbar_arrive(&bars->o_empty[wg]);
     const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-    if (i < pat.N) {
-      __nv_bfloat16* dst =
-          p.o + ((static_cast<size_t>(it.b) * pat.N + i) * p.Hq + (it.h0 + wg)) * D;
+    const uint32_t slot = smem_addr(smem + Cfg<D>::kStageOff) + (wg * 4 + wq) * Cfg<D>::kStageSlotBytes;
+    const uint32_t row_addr = slot + lane * 128;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t pk[16];
+    for (int h = 0; h < D / 64; ++h) {
+      if (lane == 0) bulk_wait_read_all();  // the slot's previous store has read it
+      __syncwarp();
 #pragma unroll
-        for (int x = 0; x < 16; ++x)
-          pk[x] = pack_bf16x2(__uint_as_float(orr[c][2 * x]) * inv_l,
-                              __uint_as_float(orr[c][2 * x + 1]) * inv_l);
-        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
-#pragma unroll
-        for (int x = 0; x < 4; ++x) d4[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+      for (int x = 0; x < 8; ++x) {  // 16-byte chunk x holds columns 64h + 8x .. 64h + 8x + 7
+        const int c = 2 * h + (x >> 2), o = (8 * x) & 31;
+        st_shared_v4(row_addr + ((x ^ (lane & 7)) << 4),
+                     pack_bf16x2(__uint_as_float(orr[c][o]) * inv_l, __uint_as_float(orr[c][o + 1]) * inv_l),
+                     pack_bf16x2(__uint_as_float(orr[c][o + 2]) * inv_l, __uint_as_float(orr[c][o + 3]) * inv_l),
+                     pack_bf16x2(__uint_as_float(orr[c][o + 4]) * inv_l, __uint_as_float(orr[c][o + 5]) * inv_l),
+                     pack_bf16x2(__uint_as_float(orr[c][o + 6]) * inv_l, __uint_as_float(orr[c][o + 7]) * inv_l));
+      }
+      fence_proxy_async_smem();  // make the generic-proxy writes visible to the TMA engine
+      __syncwarp();
+      if (lane == 0 && it.qb * BM + wq * 32 < pat.N) {  // a slot wholly past N stores nothing
+        tma_store_4d(to, slot, 64 * h, it.h0 + wg, it.qb * BM + wq * 32, it.b);
+        bulk_commit_group();
       }
     }
   }
@@ -530,7 +591,8 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                const __grid_constant__ CUtensorMap tv, const __grid_constant__ AttnParams p) {
+                const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
+                const __grid_constant__ AttnParams p) {
   constexpr int NST = Cfg<D>::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -563,6 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tq);
     tma_prefetch_desc(&tk);
     tma_prefetch_desc(&tv);
+    tma_prefetch_desc(&to);
   }
   tc_fence_before();
   __syncthreads();
@@ -571,7 +634,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 8) {
     setmaxnreg_inc<kSoftmaxRegs>();
-    softmax_role<D>(p, bars, warp >> 2, warp & 3, lane, tmem_base);
+    softmax_role<D>(p, bars, smem, &to, warp >> 2, warp & 3, lane, tmem_base);
+    if (lane == 0) bulk_wait_all();  // output stores done before shared memory goes away
+    __syncwarp();
   } else {
     setmaxnreg_dec<kSideRegs>();
   }
@@ -846,18 +911,17 @@ int launch_attention_d(const LaunchArgs& a, DeviceInfo* di) {
       return TM_ERR_CUDA;
     di->attr_set[kidx] = true;
   }
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (encode_bnhd(&tq, a.q, a.B, a.N, a.Hq, D, BM) || encode_bnhd(&tk, a.k, a.B, a.N, a.Hkv, D, BN) ||
-      encode_bnhd(&tv, a.v, a.B, a.N, a.Hkv, D, BN))
+      encode_bnhd(&tv, a.v, a.B, a.N, a.Hkv, D, BN) || encode_bnhd(&to, a.o, a.B, a.N, a.Hq, D, 32))
     return TM_ERR_CUDA;
 
   AttnParams p;
   p.sl2 = a.scale * 1.4426950408889634f;
-  p.o = static_cast<__nv_bfloat16*>(a.o);
 
   const int grid = build_schedule(a.B, a.Hq, a.Hkv, a.N, a.pat, di->sms, &p);
   attn_kernel<D><<<grid, kThreads, Cfg<D>::kSmemBytes, static_cast<cudaStream_t>(a.stream)>>>(
-      tq, tk, tv, p);
+      tq, tk, tv, to, p);
   return cudaGetLastError() == cudaSuccess ? TM_OK : TM_ERR_CUDA;
 }
 
@@ -877,11 +941,16 @@ int debug_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
   const int grid = build_schedule(B, Hq, Hkv, N, pat, max_ctas, &p);
   long long n = 0;
   for (int c = 0; c < grid; ++c) {
-    const int nw = work_count(p, c, grid);
-    for (int k = 0; k < nw; ++k, ++n) {
-      if (n >= cap) continue;
+    WorkCursor cur;
+    cur.init(p, c, grid);
+    if (cur.n_work != work_count(p, c, grid)) return TM_ERR_INVALID_ARG;
+    for (int k = 0; !cur.done(); ++k, ++n) {
+      const Item it = cur.next(p);  // what the kernel's roles see
       const int item = work_item(p, c, grid, k);
-      const Item it = decode_item(p.B, p.Hkv, p.G, p.npairs, p.nqb, p.units, item);
+      const Item ref = decode_item(p.B, p.Hkv, p.G, p.npairs, p.nqb, p.units, item);
+      if (it.qb != ref.qb || it.b != ref.b || it.g != ref.g || it.h0 != ref.h0 || it.v1 != ref.v1)
+        return TM_ERR_INVALID_ARG;  // the cursor and the direct decode disagree
+      if (n >= cap) continue;
       int* r = out + 5 * n;
       r[0] = c; r[1] = item; r[2] = it.qb; r[3] = it.b * Hq + it.h0; r[4] = 1 + it.v1;
     }
