@@ -115,7 +115,7 @@ template <int NST>
 struct Bars {
   uint64_t q_full, q_empty;
   uint64_t kv_full[NST], kv_empty[NST];
-  uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t s_full[2], p_full[4], o_full[2], o_empty[2];  // p_full[2w + h]: half h of P_w
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -264,11 +264,11 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_lo, uint32_
 // O[128 x D] (+)= P[128 x 128] (bf16 in TMEM, 2 per column) . V[128 x D];
 // V is MN-major (D contiguous per key row): 16 keys per step = 16 rows = 2048
 // bytes. v_lo: low descriptor word of the V tile (LBO = one panel).
-template <int D>
+template <int D, int K0 = 0, int K1 = BN / 16>
 __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_lo,
                                          uint32_t accumulate) {
 #pragma unroll
-  for (int kk = 0; kk < BN / 16; ++kk) {
+  for (int kk = K0; kk < K1; ++kk) {
     mma_ts(d_tmem, p_tmem + kk * 8, desc_join(v_lo + kk * (2048 >> 4), kDescHiSw128),
            Cfg<D>::kIdescO, (accumulate || kk > 0) ? 1u : 0u);
   }
@@ -392,8 +392,10 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStag
         ++oe0;
       }
       TM_WAIT(&bars->p_full[0], pc0 & 1u, kSitePFull);
+      issue_pv<D, 0, 4>(tO0, tS0, v_lo0 + vst * kStageLo, t > 0 ? 1u : 0u);
+      TM_WAIT(&bars->p_full[1], pc0 & 1u, kSitePFull);
       ++pc0;
-      issue_pv<D>(tO0, tS0, v_lo0 + vst * kStageLo, t > 0 ? 1u : 0u);
+      issue_pv<D, 4, 8>(tO0, tS0, v_lo0 + vst * kStageLo, 1u);
       if (t == T - 1) mma_commit(&bars->o_full[0]);
       if (t + 1 < T) {
         const uint32_t kidx = kv_cnt + 1;
@@ -408,9 +410,11 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStag
           TM_WAIT(&bars->o_empty[1], (oe1 & 1u) ^ 1u, kSiteOEmpty);
           ++oe1;
         }
-        TM_WAIT(&bars->p_full[1], pc1 & 1u, kSitePFull);
+        TM_WAIT(&bars->p_full[2], pc1 & 1u, kSitePFull);
+        issue_pv<D, 0, 4>(tO1, tS1, v_lo0 + vst * kStageLo, t > 0 ? 1u : 0u);
+        TM_WAIT(&bars->p_full[3], pc1 & 1u, kSitePFull);
         ++pc1;
-        issue_pv<D>(tO1, tS1, v_lo0 + vst * kStageLo, t > 0 ? 1u : 0u);
+        issue_pv<D, 4, 8>(tO1, tS1, v_lo0 + vst * kStageLo, 1u);
         if (t == T - 1) mma_commit(&bars->o_full[1]);
       }
       mma_commit(&bars->kv_empty[vst]);  // V_t free once both P.V products are done
@@ -507,9 +511,23 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
         m_run = m_new;
       }
       const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
+      // O must be rescaled before the first half of this tile's P.V is issued
+      if (t > 0 && __any_sync(0xffffffffu, bump)) {
+#pragma unroll 1
+        for (int c = 0; c < D / 16; ++c) {  // 16 columns at a time: the scores are still live
+          uint32_t orr[16];
+          tmem_ld16(tO + 16 * c, orr);
+          tmem_wait_ld16(orr);
+#pragma unroll
+          for (int x = 0; x < 16; ++x) orr[x] = __float_as_uint(__uint_as_float(orr[x]) * alpha);
+          tmem_st16(tO + 16 * c, orr);
+        }
+      }
       // p = 2^(s * scale * log2 e - m): packed fp32x2 FMA, then exp2; l sums the
       // same bf16-rounded weights that P.V uses (exact widening adds), so O / l is
-      // a properly normalised average of v (a single dominant key returns v exactly)
+      // a properly normalised average of v (a single dominant key returns v exactly).
+      // P is published in two halves (keys 0-63, 64-127): the MMA issuer starts
+      // the first half of P.V while the second half is still being exponentiated.
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -525,23 +543,12 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
           add_bf16x2_to_f32(acc[2 * (x & 3)], acc[2 * (x & 3) + 1], pk[x]);
         }
         tmem_st32(tS + 32 * h, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->p_full[2 * wg + h]);
       }
       const float rs = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
       l_run = l_run * alpha + rs;
-      if (t > 0 && __any_sync(0xffffffffu, bump)) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t orr[32];
-          tmem_ld32(tO + 32 * c, orr);
-          tmem_wait_ld(orr);
-#pragma unroll
-          for (int x = 0; x < 32; ++x) orr[x] = __float_as_uint(__uint_as_float(orr[x]) * alpha);
-          tmem_st32(tO + 32 * c, orr);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bars->p_full[wg]);
     }
     // epilogue: O / l -> bf16 -> this warp's 128B-swizzled staging slot (32 rows x
     // 64 columns at a time) -> one TMA store per half; rows past N are clipped.
@@ -608,7 +615,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&bars->s_full[w], 1);
-      mbar_init(&bars->p_full[w], 128);
+      mbar_init(&bars->p_full[2 * w], 128);
+      mbar_init(&bars->p_full[2 * w + 1], 128);
       mbar_init(&bars->o_full[w], 1);
       mbar_init(&bars->o_empty[w], 128);
     }
