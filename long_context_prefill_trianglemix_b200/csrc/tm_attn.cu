@@ -125,10 +125,14 @@ struct AttnParams {
   int B, Hq, Hkv, N, G, npairs, nqb, units;
   Pattern pat;
   float sl2;  // softmax scale * log2(e)
+  // Items: the n_hqb heaviest q-blocks (the last-L blocks of the triangle) form
+  // the big items [0, n_big = n_hqb * units), q-block major; the other items
+  // follow in (batch, kv head) major order, q-block descending, pair fastest,
+  // so that consecutive items of a CTA share almost all of their K/V tiles.
   // Work of CTA c: the big items c, c + grid, c + 2 grid, ... below n_big (dealt
   // round-robin, longest first), then the contiguous run [run_begin[c],
   // run_begin[c + 1]) of the remaining items.
-  int n_big;
+  int n_hqb, n_big;
   int run_begin[kMaxCtas + 1];
 };
 
@@ -146,19 +150,28 @@ struct Item {
   int b, g, qb, h0, v1;
 };
 
-__host__ __device__ __forceinline__ Item decode_item(int B, int Hkv, int G, int npairs, int nqb,
-                                                     int units, int item) {
-  (void)B;
+__host__ __device__ __forceinline__ Item decode_item(const AttnParams& p, int item) {
   Item it;
-  const int qi = item / units;
-  const int u = item - qi * units;
-  it.qb = nqb - 1 - qi;  // longest q-blocks first
-  const int pr = u % npairs;
-  const int gb = u / npairs;
-  it.g = gb % Hkv;
-  it.b = gb / Hkv;
-  it.h0 = it.g * G + 2 * pr;
-  it.v1 = (2 * pr + 1 < G) ? 1 : 0;
+  int pr, gb;
+  if (item < p.n_big) {  // heavy q-blocks, q-block major, longest first
+    const int qi = item / p.units;
+    const int u = item - qi * p.units;
+    it.qb = p.nqb - 1 - qi;
+    pr = u % p.npairs;
+    gb = u / p.npairs;
+  } else {  // (batch, kv head) major, q-block descending, pair fastest
+    const int j = item - p.n_big;
+    const int nq = p.nqb - p.n_hqb;
+    pr = j % p.npairs;
+    const int r = j / p.npairs;
+    const int qi = r % nq;
+    gb = r / nq;
+    it.qb = nq - 1 - qi;
+  }
+  it.g = gb % p.Hkv;
+  it.b = gb / p.Hkv;
+  it.h0 = it.g * p.G + 2 * pr;
+  it.v1 = (2 * pr + 1 < p.G) ? 1 : 0;
   return it;
 }
 
@@ -169,18 +182,19 @@ __host__ __device__ __forceinline__ Item decode_item(int B, int Hkv, int G, int 
 // batch -> q-block with carries.
 struct WorkCursor {
   int k, n_work, nb, big_next, g;
-  int qi, pr, kvh, b;  // position of the next run item
+  int pr, qi, kvh, b;  // position of the next run item
   __host__ __device__ __forceinline__ void init(const AttnParams& p, int c, int grid) {
     g = grid;
     nb = c < p.n_big ? (p.n_big - c + g - 1) / g : 0;
     n_work = nb + p.run_begin[c + 1] - p.run_begin[c];
     k = 0;
     big_next = c;
-    const int item = p.run_begin[c];
-    qi = item / p.units;
-    const int u = item - qi * p.units;
-    pr = u % p.npairs;
-    const int gb = u / p.npairs;
+    const int j = p.run_begin[c] - p.n_big;  // runs cover the non-big items only
+    const int nq = p.nqb - p.n_hqb;
+    pr = j % p.npairs;
+    const int r = j / p.npairs;
+    qi = nq > 0 ? r % nq : 0;
+    const int gb = nq > 0 ? r / nq : 0;
     kvh = gb % p.Hkv;
     b = gb / p.Hkv;
   }
@@ -189,21 +203,21 @@ struct WorkCursor {
   __host__ __device__ __forceinline__ Item next(const AttnParams& p) {
     Item it;
     if (k < nb) {
-      it = decode_item(p.B, p.Hkv, p.G, p.npairs, p.nqb, p.units, big_next);
+      it = decode_item(p, big_next);
       big_next += g;
     } else {
-      it.qb = p.nqb - 1 - qi;
+      it.qb = p.nqb - p.n_hqb - 1 - qi;
       it.g = kvh;
       it.b = b;
       it.h0 = kvh * p.G + 2 * pr;
       it.v1 = (2 * pr + 1 < p.G) ? 1 : 0;
       if (++pr == p.npairs) {
         pr = 0;
-        if (++kvh == p.Hkv) {
-          kvh = 0;
-          if (++b == p.B) {
-            b = 0;
-            ++qi;
+        if (++qi == p.nqb - p.n_hqb) {
+          qi = 0;
+          if (++kvh == p.Hkv) {
+            kvh = 0;
+            ++b;
           }
         }
       }
@@ -537,8 +551,13 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
           // the first kPolyPairs pairs of every 32 use the FMA-pipe exp2, the rest MUFU
           float xa, xb;
           ffma2(xa, xb, s[64 * h + 2 * x], s[64 * h + 2 * x + 1], sl2, sl2, neg_m, neg_m);
-          const float a = x < kPolyPairs ? ex2_poly(xa) : ex2(xa);
-          const float b = x < kPolyPairs ? ex2_poly(xb) : ex2(xb);
+          float a, b;
+          if (x < kPolyPairs) {
+            ex2x2_poly(a, b, xa, xb);
+          } else {
+            a = ex2(xa);
+            b = ex2(xb);
+          }
           pk[x] = pack_bf16x2(a, b);
           add_bf16x2_to_f32(acc[2 * (x & 3)], acc[2 * (x & 3) + 1], pk[x]);
         }
@@ -864,12 +883,20 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
     total += qcost[qb] * static_cast<long long>(B) * Hq;
   }
   auto item_cost = [&](long long item) {
-    const Item it = decode_item(p->B, p->Hkv, p->G, p->npairs, p->nqb, p->units, static_cast<int>(item));
+    const Item it = decode_item(*p, static_cast<int>(item));
     return qcost[it.qb] * (1 + it.v1);
   };
   const double target = static_cast<double>(total) / grid;
-  long long n_big = 0;
-  while (n_big < n_items && n_big < 8LL * grid && 4.0 * item_cost(n_big) > target) ++n_big;
+  // heavy q-blocks: from the top, while an item of the block costs more than a
+  // quarter of a CTA's share (at most 8 big items per CTA)
+  const long long item_q = qcost.empty() ? 0 : (p->G >= 2 ? 2 : 1);
+  int n_hqb = 0;
+  while (n_hqb < p->nqb - 1 && 4.0 * qcost[p->nqb - 1 - n_hqb] * item_q > target &&
+         static_cast<long long>(n_hqb + 1) * p->units <= 8LL * grid)
+    ++n_hqb;
+  p->n_hqb = n_hqb;
+  p->n_big = n_hqb * p->units;
+  const long long n_big = p->n_big;
   std::vector<double> cap(grid, target);
   double big_total = 0;
   for (long long j = 0; j < n_big; ++j) {
@@ -880,7 +907,6 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
   double cap_total = 0;
   for (int c = 0; c < grid; ++c) cap_total += std::max(0.0, cap[c]);
   const double rest = static_cast<double>(total) - big_total;
-  p->n_big = static_cast<int>(n_big);
   p->run_begin[0] = static_cast<int>(n_big);
   int c = 0;
   double acc = 0, bound = 0;
@@ -955,7 +981,7 @@ int debug_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
     for (int k = 0; !cur.done(); ++k, ++n) {
       const Item it = cur.next(p);  // what the kernel's roles see
       const int item = work_item(p, c, grid, k);
-      const Item ref = decode_item(p.B, p.Hkv, p.G, p.npairs, p.nqb, p.units, item);
+      const Item ref = decode_item(p, item);
       if (it.qb != ref.qb || it.b != ref.b || it.g != ref.g || it.h0 != ref.h0 || it.v1 != ref.v1)
         return TM_ERR_INVALID_ARG;  // the cursor and the direct decode disagree
       if (n >= cap) continue;

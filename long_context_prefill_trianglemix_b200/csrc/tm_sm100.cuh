@@ -320,6 +320,36 @@ __device__ __forceinline__ float ex2_poly(float x) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
+// Two exponentials 2^xa, 2^xb with packed fp32x2 arithmetic (same method as
+// ex2_poly): clamp at -125, n = round(x) through the 1.5 * 2^23 shift, f = x - n,
+// 2^f by the fitted cubic in three packed FMAs, and 2^n added to the exponent
+// field with one integer multiply-add per value.
+__device__ __forceinline__ void ex2x2_poly(float& ra, float& rb, float xa, float xb) {
+  xa = fmaxf(xa, -125.0f);
+  xb = fmaxf(xb, -125.0f);
+  uint32_t ta, tb, pa, pb;
+  asm("{\n\t.reg .b64 x, m, t, n, f, p, c;\n\t"
+      "mov.b64 x, {%4, %5};\n\t"
+      "mov.b64 m, {%6, %6};\n\t"
+      "add.rn.f32x2 t, x, m;\n\t"           // round to an integer in the low mantissa bits
+      "sub.rn.f32x2 n, t, m;\n\t"
+      "sub.rn.f32x2 f, x, n;\n\t"           // f in [-1/2, 1/2]
+      "mov.b64 c, {%7, %7};\n\t"
+      "mov.b64 p, {%8, %8};\n\t"
+      "fma.rn.f32x2 p, c, f, p;\n\t"
+      "mov.b64 c, {%9, %9};\n\t"
+      "fma.rn.f32x2 p, p, f, c;\n\t"
+      "mov.b64 c, {%10, %10};\n\t"
+      "fma.rn.f32x2 p, p, f, c;\n\t"
+      "mov.b64 {%0, %1}, t;\n\t"
+      "mov.b64 {%2, %3}, p;\n\t}"
+      : "=r"(ta), "=r"(tb), "=r"(pa), "=r"(pb)
+      : "f"(xa), "f"(xb), "f"(12582912.0f), "f"(TM_EXP2_C3), "f"(TM_EXP2_C2), "f"(TM_EXP2_C1),
+        "f"(TM_EXP2_C0));
+  ra = __uint_as_float(ta * 8388608u + pa);  // the integer n sits in t's low bits
+  rb = __uint_as_float(tb * 8388608u + pb);
+}
+
 // (d0, d1) = (a0, a1) * (b0, b1) + (c0, c1) as one packed fp32x2 FMA.
 __device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
                                       float c0, float c1) {

@@ -50,10 +50,25 @@ def test_triangle_split_is_balanced(N, S, W, L):
     cost = np.zeros(148)
     for c, item, qb, h0, nv in rec:
         cost[c] += (per_qb[qb] + 3) * nv
-    # within one normal item of the mean, and big items first in each CTA
+    # within one normal item of the mean
     normal = (per_qb[:-3].max() + 3) * 2
     assert cost.max() - cost.mean() <= 1.5 * normal, (cost.max(), cost.mean(), normal)
+    # a CTA's big items (the last-L q-blocks) come before its other items
+    heavy = set(np.flatnonzero(per_qb >= 4 * normal).tolist())
+    assert heavy, "the last-L q-blocks are big items"
     for c in range(148):
-        qbs = rec[rec[:, 0] == c][:, 2]
-        costs = per_qb[qbs]
-        assert costs[0] == costs.max()
+        qbs = rec[rec[:, 0] == c][:, 2].tolist()
+        flags = [q in heavy for q in qbs]
+        assert flags == sorted(flags, reverse=True), (c, qbs[:6])
+
+
+def test_consecutive_items_share_kv_tiles():
+    # after the big items, a CTA walks one kv head's q-blocks downwards, pair by pair
+    rec = tm.tm_debug_schedule(1, 32, 8, 32768, False, 64, 1024, 128, 148)
+    for c in range(148):
+        r = rec[rec[:, 0] == c]
+        r = r[r[:, 2] < 255]
+        kvh = (r[:, 3] % 32) // 4
+        same = (np.diff(kvh) == 0)
+        step = np.diff(r[:, 2])
+        assert np.all(step[same] <= 0) and np.all(step[same] >= -1)
