@@ -36,9 +36,11 @@ from long_context_prefill_trianglemix_b200 import inputs as I  # noqa: E402
 METRIC = "triangle-attn prefill TFLOP/s (kept tiles) at 128K; speedup vs own causal"
 UNIT = "TFLOP/s"
 BM = BN = 128
-# Per-launch DRAM traffic of the triangle kernel from an ncu capture, keyed by
-# the hash of the kernel sources it was taken on (reported only while they match).
-TRAFFIC = {}
+# Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the
+# triangle launch of the default workload (llama3-8b-128k, W=2048) from one ncu
+# capture of this bench command, keyed by the hash of the kernel sources it was
+# taken on; reported only while the sources still match (else null).
+TRAFFIC = {"1807816c69e24010": 2.30e9 + 1.04e9}
 
 
 def kernel_source_hash() -> str:
@@ -149,6 +151,22 @@ def oracle_sample(wl, W, n_rows: int, seed: int, host, target_s: float = 0.0):
 
 
 # ----------------------------------------------------------------------------- arms
+
+def reduce_over_ranks(values, device="cpu"):
+    """Max over ranks of per-rank timings (ms). The replicas share no data: this
+    reduction of the timings is the only collective of a multi-GPU run."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_tflops(n_ranks, steps, flop_per_step, max_ms_total):
+    """Throughput of N replicas: all ranks' work over the slowest rank's time."""
+    return n_ranks * steps * flop_per_step / (max_ms_total * 1e-3) / 1e12
+
 
 def dist_setup():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
@@ -267,15 +285,12 @@ def run_ours(args):
     torch.cuda.synchronize()
     e2e_ms = sum(ee[s][0].elapsed_time(ee[s][1]) for s in range(e2e_steps)) / e2e_steps
 
-    if ws > 1:
-        t = torch.tensor([total_ms, tri_sum, e2e_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, tri_sum, e2e_ms = t.tolist()
+    total_ms, tri_sum, e2e_ms = reduce_over_ranks([total_ms, tri_sum, e2e_ms], device="cuda")
 
     peaks = load_peaks()
     tri_avg = tri_sum / args.steps
     achieved = tri_f / (tri_avg * 1e-3) / 1e12
-    value = ws * args.steps * tri_f / (tri_sum * 1e-3) / 1e12
+    value = whole_job_tflops(ws, args.steps, tri_f, tri_sum)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -299,7 +314,7 @@ def run_ours(args):
                                   "a long step after the causal layer)",
                      "frac_of_burst": achieved / peaks["burst"],
                      "traffic": TRAFFIC.get(kernel_source_hash())},
-        "e2e": {"value": ws * tri_f / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+        "e2e": {"value": whole_job_tflops(ws, 1, tri_f, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": int((dq.numel() + dk.numel() + dv.numel()) * 2),
                 "d2h_bytes_per_step": int(do.numel() * 2),
                 "what": "pinned host q,k,v -> device, triangle layer, output -> pinned host"},

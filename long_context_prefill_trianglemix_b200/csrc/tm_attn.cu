@@ -125,25 +125,48 @@ struct AttnParams {
   int B, Hq, Hkv, N, G, npairs, nqb, units;
   Pattern pat;
   float sl2;  // softmax scale * log2(e)
-  // Items: the n_hqb heaviest q-blocks (the last-L blocks of the triangle) form
-  // the big items [0, n_big = n_hqb * units), q-block major; the other items
-  // follow in (batch, kv head) major order, q-block descending, pair fastest,
-  // so that consecutive items of a CTA share almost all of their K/V tiles.
-  // Work of CTA c: the big items c, c + grid, c + 2 grid, ... below n_big (dealt
-  // round-robin, longest first), then the contiguous run [run_begin[c],
-  // run_begin[c + 1]) of the remaining items.
-  int n_hqb, n_big;
-  int run_begin[kMaxCtas + 1];
+  // Items run q-block major (longest q-blocks first), the (batch, kv head,
+  // pair) units inside. The first n_big items (the n_hqb heaviest q-blocks, the
+  // last-L blocks of the triangle) are dealt round-robin: CTA c takes c,
+  // c + grid, ... Every other item is dealt in strided rounds, so that the CTAs
+  // running at the same time work on neighbouring q-blocks of every kv head and
+  // each K/V tile is read from DRAM about once per round. The first n_a CTAs
+  // hold one big item more than the rest and join the rounds n_skip rounds
+  // late. Normal item j of CTA c (j counted from 0):
+  //   c >= n_a and j < n_skip:  (c - n_a) + j * (grid - n_a)
+  //   otherwise:                 n_skip * (grid - n_a) + (j - s_c) * grid + c,
+  //                              s_c = n_skip if c >= n_a else 0
+  int n_hqb, n_big, n_a, n_skip;
 };
 
+__host__ __device__ __forceinline__ int big_count(const AttnParams& p, int c, int g) {
+  return c < p.n_big ? (p.n_big - c + g - 1) / g : 0;
+}
+
+// Normal index (counted from 0 after the big items) of CTA c's j-th normal item.
+__host__ __device__ __forceinline__ long long normal_index(const AttnParams& p, int c, int g, int j) {
+  const int ga = g - p.n_a;
+  if (c >= p.n_a) {
+    if (j < p.n_skip) return static_cast<long long>(c - p.n_a) + static_cast<long long>(j) * ga;
+    return static_cast<long long>(p.n_skip) * ga + static_cast<long long>(j - p.n_skip) * g + c;
+  }
+  return static_cast<long long>(p.n_skip) * ga + static_cast<long long>(j) * g + c;
+}
+
 __host__ __device__ __forceinline__ int work_count(const AttnParams& p, int c, int g) {
-  const int nb = c < p.n_big ? (p.n_big - c + g - 1) / g : 0;
-  return nb + p.run_begin[c + 1] - p.run_begin[c];
+  const long long n_norm = static_cast<long long>(p.nqb) * p.units - p.n_big;
+  // largest j with normal_index(j) < n_norm, + 1 (monotone in j)
+  int lo = 0, hi = static_cast<int>(n_norm) + 1;
+  while (lo < hi) {
+    const int mid = (lo + hi) / 2;
+    if (normal_index(p, c, g, mid) < n_norm) lo = mid + 1; else hi = mid;
+  }
+  return big_count(p, c, g) + lo;
 }
 
 __host__ __device__ __forceinline__ int work_item(const AttnParams& p, int c, int g, int k) {
-  const int nb = c < p.n_big ? (p.n_big - c + g - 1) / g : 0;
-  return k < nb ? c + k * g : p.run_begin[c] + (k - nb);
+  const int nb = big_count(p, c, g);
+  return k < nb ? c + k * g : p.n_big + static_cast<int>(normal_index(p, c, g, k - nb));
 }
 
 struct Item {
@@ -152,22 +175,11 @@ struct Item {
 
 __host__ __device__ __forceinline__ Item decode_item(const AttnParams& p, int item) {
   Item it;
-  int pr, gb;
-  if (item < p.n_big) {  // heavy q-blocks, q-block major, longest first
-    const int qi = item / p.units;
-    const int u = item - qi * p.units;
-    it.qb = p.nqb - 1 - qi;
-    pr = u % p.npairs;
-    gb = u / p.npairs;
-  } else {  // (batch, kv head) major, q-block descending, pair fastest
-    const int j = item - p.n_big;
-    const int nq = p.nqb - p.n_hqb;
-    pr = j % p.npairs;
-    const int r = j / p.npairs;
-    const int qi = r % nq;
-    gb = r / nq;
-    it.qb = nq - 1 - qi;
-  }
+  const int qi = item / p.units;
+  const int u = item - qi * p.units;
+  it.qb = p.nqb - 1 - qi;  // longest q-blocks first
+  const int pr = u % p.npairs;
+  const int gb = u / p.npairs;
   it.g = gb % p.Hkv;
   it.b = gb / p.Hkv;
   it.h0 = it.g * p.G + 2 * pr;
@@ -175,28 +187,47 @@ __host__ __device__ __forceinline__ Item decode_item(const AttnParams& p, int it
   return it;
 }
 
-// Walks one CTA's work (the same sequence as work_item) without integer
-// division per item: an integer division costs a MUFU reciprocal, and MUFU is
-// the unit the softmax warps keep busy with exp2. Big items are decoded
-// directly (a few per CTA); the contiguous run advances pair -> kv head ->
-// batch -> q-block with carries.
+// Walks one CTA's work (the same sequence as work_item) without an integer
+// division per item: a division costs a MUFU reciprocal, and MUFU is the unit
+// the softmax warps keep busy with exp2. Within each strided phase the item
+// index grows by a fixed stride, added digit by digit in the mixed radix
+// (pair, kv head, batch | q-block) of the item index.
 struct WorkCursor {
-  int k, n_work, nb, big_next, g;
-  int pr, qi, kvh, b;  // position of the next run item
-  __host__ __device__ __forceinline__ void init(const AttnParams& p, int c, int grid) {
-    g = grid;
-    nb = c < p.n_big ? (p.n_big - c + g - 1) / g : 0;
-    n_work = nb + p.run_begin[c + 1] - p.run_begin[c];
-    k = 0;
-    big_next = c;
-    const int j = p.run_begin[c] - p.n_big;  // runs cover the non-big items only
-    const int nq = p.nqb - p.n_hqb;
-    pr = j % p.npairs;
-    const int r = j / p.npairs;
-    qi = nq > 0 ? r % nq : 0;
-    const int gb = nq > 0 ? r / nq : 0;
+  int k, n_work, nb, big_next, g, c;
+  int j, phase_end;                 // normal position; where the current stride ends
+  int pr, kvh, b, qi;               // digits of the next normal item
+  int d_pr, d_kvh, d_b, d_qi;       // digits of the current stride
+  __host__ __device__ __forceinline__ void set_item(const AttnParams& p, long long item) {
+    qi = static_cast<int>(item / p.units);
+    const int u = static_cast<int>(item - static_cast<long long>(qi) * p.units);
+    pr = u % p.npairs;
+    const int gb = u / p.npairs;
     kvh = gb % p.Hkv;
     b = gb / p.Hkv;
+  }
+  __host__ __device__ __forceinline__ void set_stride(const AttnParams& p, int stride) {
+    d_qi = stride / p.units;
+    const int u = stride - d_qi * p.units;
+    d_pr = u % p.npairs;
+    const int gb = u / p.npairs;
+    d_kvh = gb % p.Hkv;
+    d_b = gb / p.Hkv;
+  }
+  __host__ __device__ __forceinline__ void enter_phase(const AttnParams& p) {
+    set_item(p, p.n_big + normal_index(p, c, g, j));
+    const bool late = c >= p.n_a && j < p.n_skip;
+    set_stride(p, late ? g - p.n_a : g);
+    phase_end = late ? p.n_skip : 0x7fffffff;
+  }
+  __host__ __device__ __forceinline__ void init(const AttnParams& p, int cta, int grid) {
+    c = cta;
+    g = grid;
+    nb = big_count(p, c, g);
+    n_work = work_count(p, c, g);
+    k = 0;
+    big_next = c;
+    j = 0;
+    enter_phase(p);
   }
   __host__ __device__ __forceinline__ bool done() const { return k >= n_work; }
   // Returns the next item of this CTA and advances.
@@ -206,20 +237,25 @@ struct WorkCursor {
       it = decode_item(p, big_next);
       big_next += g;
     } else {
-      it.qb = p.nqb - p.n_hqb - 1 - qi;
+      it.qb = p.nqb - 1 - qi;
       it.g = kvh;
       it.b = b;
       it.h0 = kvh * p.G + 2 * pr;
       it.v1 = (2 * pr + 1 < p.G) ? 1 : 0;
-      if (++pr == p.npairs) {
-        pr = 0;
-        if (++qi == p.nqb - p.n_hqb) {
-          qi = 0;
-          if (++kvh == p.Hkv) {
-            kvh = 0;
-            ++b;
-          }
-        }
+      ++j;
+      if (j == phase_end) {
+        enter_phase(p);
+      } else {  // add the stride digit by digit
+        int carry = 0;
+        pr += d_pr;
+        if (pr >= p.npairs) { pr -= p.npairs; carry = 1; }
+        kvh += d_kvh + carry;
+        carry = 0;
+        if (kvh >= p.Hkv) { kvh -= p.Hkv; carry = 1; }
+        b += d_b + carry;
+        carry = 0;
+        if (b >= p.B) { b -= p.B; carry = 1; }
+        qi += d_qi + carry;
       }
     }
     ++k;
@@ -870,10 +906,9 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
   p->units = B * Hkv * p->npairs;
   p->pat = pat;
   // Persistent grid. Item cost = (visited tiles + fixed per-item overhead,
-  // about the pipeline fill/drain and epilogue) x Q tiles of the item. Items
-  // costing more than a quarter of a CTA's share (the last-L q-blocks of the
-  // triangle) are dealt round-robin first, longest first; the rest are split
-  // into contiguous runs sized by what each CTA still has room for.
+  // about the pipeline fill/drain and epilogue) x Q tiles of the item; it is
+  // used to find the heavy q-blocks and how many rounds the CTAs holding an
+  // extra heavy item sit out.
   const long long n_items = static_cast<long long>(p->nqb) * p->units;
   const int grid = static_cast<int>(std::min<long long>(std::min(max_ctas, kMaxCtas), n_items));
   std::vector<long long> qcost(p->nqb);
@@ -882,47 +917,32 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
     qcost[qb] = block_tiles(p->pat, qb, BM, BN).count() + kItemOverheadTiles;
     total += qcost[qb] * static_cast<long long>(B) * Hq;
   }
-  auto item_cost = [&](long long item) {
-    const Item it = decode_item(*p, static_cast<int>(item));
-    return qcost[it.qb] * (1 + it.v1);
-  };
   const double target = static_cast<double>(total) / grid;
   // heavy q-blocks: from the top, while an item of the block costs more than a
   // quarter of a CTA's share (at most 8 big items per CTA)
-  const long long item_q = qcost.empty() ? 0 : (p->G >= 2 ? 2 : 1);
+  const long long item_q = p->G >= 2 ? 2 : 1;
   int n_hqb = 0;
   while (n_hqb < p->nqb - 1 && 4.0 * qcost[p->nqb - 1 - n_hqb] * item_q > target &&
          static_cast<long long>(n_hqb + 1) * p->units <= 8LL * grid)
     ++n_hqb;
   p->n_hqb = n_hqb;
   p->n_big = n_hqb * p->units;
-  const long long n_big = p->n_big;
-  std::vector<double> cap(grid, target);
-  double big_total = 0;
-  for (long long j = 0; j < n_big; ++j) {
-    const double c = static_cast<double>(item_cost(j));
-    cap[j % grid] -= c;
-    big_total += c;
+  p->n_a = 0;
+  p->n_skip = 0;
+  const long long n_norm = n_items - p->n_big;
+  if (p->n_big % grid != 0 && n_norm > 0) {
+    // CTAs [0, n_a) hold one big item more; they sit out the rounds that the
+    // others spend on an equal cost of normal items
+    double big_cost = 0, norm_cost = 0;
+    for (int q = 0; q < n_hqb; ++q) big_cost += qcost[p->nqb - 1 - q];
+    big_cost = big_cost * B * Hq / p->n_big;
+    for (int qb = 0; qb < p->nqb - n_hqb; ++qb) norm_cost += qcost[qb];
+    norm_cost = norm_cost * B * Hq / n_norm;
+    p->n_a = p->n_big % grid;
+    const double rounds = big_cost / norm_cost;
+    const long long max_rounds = n_norm / std::max(1, grid - p->n_a);
+    p->n_skip = static_cast<int>(std::min<long long>(max_rounds, static_cast<long long>(rounds + 0.5)));
   }
-  double cap_total = 0;
-  for (int c = 0; c < grid; ++c) cap_total += std::max(0.0, cap[c]);
-  const double rest = static_cast<double>(total) - big_total;
-  p->run_begin[0] = static_cast<int>(n_big);
-  int c = 0;
-  double acc = 0, bound = 0;
-  auto next_bound = [&](int cc) {
-    return cap_total > 0 ? bound + rest * std::max(0.0, cap[cc]) / cap_total : rest * (cc + 1) / grid;
-  };
-  bound = next_bound(0);
-  for (long long item = n_big; item < n_items; ++item) {
-    while (c + 1 < grid && acc >= bound) {
-      p->run_begin[++c] = static_cast<int>(item);
-      bound = next_bound(c);
-    }
-    acc += static_cast<double>(item_cost(item));
-  }
-  while (c + 1 <= grid) p->run_begin[++c] = static_cast<int>(n_items);
-
   return grid;
 }
 
