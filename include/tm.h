@@ -22,7 +22,8 @@
  * Ownership and threading:
  *   - q, k, v, o are DEVICE pointers owned by the caller, 16-byte aligned;
  *     o must not overlap q, k or v. The library allocates no device memory
- *     in any call and keeps no per-call state.
+ *     in any call and keeps no per-call state; scratch for the split
+ *     schedule is a caller-owned workspace (the *_ws calls).
  *   - `stream` is a cudaStream_t (CUstream) handle passed as void*; NULL is
  *     the legacy default stream. Work is enqueued asynchronously on it and
  *     the call returns without synchronising.
@@ -93,6 +94,45 @@ TM_API int tm_trianglemix_attn_fwd(const void* q, const void* k, const void* v, 
                                    int L, int layer, int tri_start, void* stream);
 
 /*
+ * Split schedule for the long q-blocks. The last L query rows of the triangle
+ * (and the last rows of causal attention) see every earlier key, so one of
+ * their items can cost more than a CTA's share of the launch when B * Hq is
+ * small (a tensor-parallel shard, one sequence). With a workspace the
+ * library cuts such items into pieces over ranges of their tile list; each
+ * piece writes its unnormalised partial output with its running row max m and
+ * row sum l, and the piece that finishes last merges them (log-sum-exp merge:
+ * O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, M = max_s m_s) in piece
+ * order, so the result is deterministic. The output equals that of the
+ * entry points without a workspace up to float rounding.
+ *
+ * tm_attn_workspace_size: bytes of workspace the *_ws calls need for this
+ * problem on a grid of num_ctas CTAs (pass 0 for the current device's SM
+ * count); 0 if nothing would be split. Host only, except that num_ctas = 0
+ * queries the device.
+ *
+ * tm_*_ws: the entry points above with a caller-owned DEVICE workspace of
+ * workspace_bytes bytes, 16-byte aligned, not overlapping q, k, v or o.
+ * workspace = NULL with workspace_bytes = 0 splits nothing (identical to the
+ * calls without _ws). A workspace smaller than tm_attn_workspace_size reports
+ * gives TM_ERR_INVALID_ARG. Each call clears the counters it uses (an async
+ * memset on `stream`) and uses the rest as scratch: calls sharing one
+ * workspace must be ordered (same stream, or synchronised); the contents are
+ * undefined afterwards.
+ */
+TM_API int tm_attn_workspace_size(int B, int Hq, int Hkv, int N, int D, int causal, int S, int W,
+                                  int L, int num_ctas, long long* bytes);
+TM_API int tm_causal_attn_fwd_ws(const void* q, const void* k, const void* v, void* o, int B,
+                                 int Hq, int Hkv, int N, int D, float scale, void* workspace,
+                                 long long workspace_bytes, void* stream);
+TM_API int tm_triangle_attn_fwd_ws(const void* q, const void* k, const void* v, void* o, int B,
+                                   int Hq, int Hkv, int N, int D, float scale, int S, int W, int L,
+                                   void* workspace, long long workspace_bytes, void* stream);
+TM_API int tm_trianglemix_attn_fwd_ws(const void* q, const void* k, const void* v, void* o, int B,
+                                      int Hq, int Hkv, int N, int D, float scale, int S, int W,
+                                      int L, int layer, int tri_start, void* workspace,
+                                      long long workspace_bytes, void* stream);
+
+/*
  * Number of kept (i, j) pairs of one (batch, head) of the triangle pattern:
  * sum over rows of min(i+1, W) + max(0, min(S, i+1-W)) for i < N-L and i+1
  * otherwise. Host only. Returns -1 on a bad argument.
@@ -141,14 +181,18 @@ TM_API int tm_debug_mma_probe(const void* q, const void* k, const void* v, float
 
 /*
  * Host export of the persistent work split the kernels use on a grid of
- * num_ctas CTAs (the SM count on a B200): one record of five ints per work
- * item, (cta, item, q-block, first q head (batch * Hq + head), number of Q
- * tiles 1 or 2), in the order each CTA processes them. An item covers one
- * q-block of one or two q heads that share a kv head. out: HOST buffer of
- * 5*cap ints (NULL when cap = 0); *count receives the total. Host only.
+ * num_ctas CTAs (the SM count on a B200); split != 0 gives the split schedule
+ * of the *_ws calls, 0 the one of the calls without workspace. One record of
+ * seven ints per work item, (cta, item, q-block, first q head
+ * (batch * Hq + head), number of Q tiles 1 or 2, first tile, end tile), in the
+ * order each CTA processes them; the tiles are positions [first, end) in the
+ * q-block's tile list (the whole list unless the item is a piece). An item
+ * covers one q-block of one or two q heads that share a kv head. out: HOST
+ * buffer of 7*cap ints (NULL when cap = 0); *count receives the total. Host
+ * only.
  */
 TM_API int tm_debug_schedule(int B, int Hq, int Hkv, int N, int causal, int S, int W, int L,
-                             int num_ctas, int* out, long long cap, long long* count);
+                             int num_ctas, int split, int* out, long long cap, long long* count);
 
 /*
  * Synchronises `stream`, then reads and clears the device status word of the

@@ -26,7 +26,8 @@ EXPORTED = (
     "tm_causal_attn_fwd", "tm_triangle_attn_fwd", "tm_trianglemix_attn_fwd",
     "tm_triangle_kept_pairs", "tm_kept_tiles", "tm_triangle_tile_list", "tm_tile_list",
     "tm_debug_dump_tiles", "tm_debug_mma_probe", "tm_debug_schedule", "tm_get_device_status",
-    "tm_status_string",
+    "tm_status_string", "tm_attn_workspace_size", "tm_causal_attn_fwd_ws", "tm_triangle_attn_fwd_ws",
+    "tm_trianglemix_attn_fwd_ws",
 )
 
 
@@ -61,8 +62,15 @@ def lib() -> ctypes.CDLL:
             "tm_tile_list": (ci, [ci, ci, ci, ci, ci, ci, ci, vp, cll, ctypes.POINTER(cll)]),
             "tm_debug_dump_tiles": (ci, [ci, ci, ci, ci, ci, vp, cll, ctypes.POINTER(cll), vp]),
             "tm_debug_mma_probe": (ci, [vp, vp, vp, vp, vp, ci, vp]),
-            "tm_debug_schedule": (ci, [ci, ci, ci, ci, ci, ci, ci, ci, ci, vp, cll,
+            "tm_debug_schedule": (ci, [ci, ci, ci, ci, ci, ci, ci, ci, ci, ci, vp, cll,
                                        ctypes.POINTER(cll)]),
+            "tm_attn_workspace_size": (ci, [ci, ci, ci, ci, ci, ci, ci, ci, ci, ci,
+                                            ctypes.POINTER(cll)]),
+            "tm_causal_attn_fwd_ws": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp, cll, vp]),
+            "tm_triangle_attn_fwd_ws": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci, ci,
+                                             vp, cll, vp]),
+            "tm_trianglemix_attn_fwd_ws": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci,
+                                                ci, ci, ci, vp, cll, vp]),
             "tm_get_device_status": (ci, [vp]),
             "tm_status_string": (ctypes.c_char_p, [ci]),
         }
@@ -119,6 +127,35 @@ def tm_trianglemix_attn_fwd(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L, layer,
         _stream(stream)))
 
 
+def tm_causal_attn_fwd_ws(q, k, v, o, B, Hq, Hkv, N, D, scale, workspace, workspace_bytes,
+                          stream=None):
+    return _check("tm_causal_attn_fwd_ws", lib().tm_causal_attn_fwd_ws(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, Hkv, N, D, scale, _ptr(workspace),
+        int(workspace_bytes), _stream(stream)))
+
+
+def tm_triangle_attn_fwd_ws(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L, workspace,
+                            workspace_bytes, stream=None):
+    return _check("tm_triangle_attn_fwd_ws", lib().tm_triangle_attn_fwd_ws(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, Hkv, N, D, scale, S, W, L, _ptr(workspace),
+        int(workspace_bytes), _stream(stream)))
+
+
+def tm_trianglemix_attn_fwd_ws(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L, layer, tri_start,
+                               workspace, workspace_bytes, stream=None):
+    return _check("tm_trianglemix_attn_fwd_ws", lib().tm_trianglemix_attn_fwd_ws(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, Hkv, N, D, scale, S, W, L, layer, tri_start,
+        _ptr(workspace), int(workspace_bytes), _stream(stream)))
+
+
+def tm_attn_workspace_size(B, Hq, Hkv, N, D, causal, S, W, L, num_ctas=0) -> int:
+    """Workspace bytes of the split schedule (0: nothing is split)."""
+    n = ctypes.c_longlong(0)
+    _check("tm_attn_workspace_size", lib().tm_attn_workspace_size(
+        B, Hq, Hkv, N, D, int(causal), S, W, L, num_ctas, ctypes.byref(n)))
+    return n.value
+
+
 def tm_triangle_kept_pairs(N, S, W, L) -> int:
     return int(lib().tm_triangle_kept_pairs(N, S, W, L))
 
@@ -160,15 +197,17 @@ def tm_debug_mma_probe(q, k, v, s_out, o_out, D, stream=None):
         _ptr(q), _ptr(k), _ptr(v), _ptr(s_out), _ptr(o_out), D, _stream(stream)))
 
 
-def tm_debug_schedule(B, Hq, Hkv, N, causal, S, W, L, num_ctas=148) -> np.ndarray:
-    """Persistent work split as an int32 [n, 5] array: (cta, item, q-block, head0, tiles)."""
+def tm_debug_schedule(B, Hq, Hkv, N, causal, S, W, L, num_ctas=148, split=False) -> np.ndarray:
+    """Persistent work split as an int32 [n, 7] array:
+    (cta, item, q-block, head0, Q tiles, first tile, end tile)."""
     cnt = ctypes.c_longlong(0)
     _check("tm_debug_schedule", lib().tm_debug_schedule(B, Hq, Hkv, N, int(causal), S, W, L,
-                                                        num_ctas, None, 0, ctypes.byref(cnt)))
-    out = np.zeros((max(cnt.value, 1), 5), np.int32)
-    _check("tm_debug_schedule", lib().tm_debug_schedule(B, Hq, Hkv, N, int(causal), S, W, L,
-                                                        num_ctas, out.ctypes.data, cnt.value,
+                                                        num_ctas, int(split), None, 0,
                                                         ctypes.byref(cnt)))
+    out = np.zeros((max(cnt.value, 1), 7), np.int32)
+    _check("tm_debug_schedule", lib().tm_debug_schedule(B, Hq, Hkv, N, int(causal), S, W, L,
+                                                        num_ctas, int(split), out.ctypes.data,
+                                                        cnt.value, ctypes.byref(cnt)))
     return out[: cnt.value]
 
 

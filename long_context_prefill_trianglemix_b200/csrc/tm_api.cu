@@ -45,13 +45,30 @@ int validate_pattern(int S, int W, int L) {
   return TM_OK;
 }
 
+// Workspace of the split entry points: NULL with 0 bytes (nothing is split),
+// or 16-byte aligned, not overlapping q, k, v or o.
+int validate_workspace(const void* q, const void* k, const void* v, const void* o, int B, int Hq,
+                       int Hkv, int N, int D, const void* ws, long long ws_bytes) {
+  if (ws_bytes < 0 || (!ws && ws_bytes != 0)) return TM_ERR_INVALID_ARG;
+  if (!ws) return TM_OK;
+  if (!aligned16(ws)) return TM_ERR_INVALID_ARG;
+  const long long rows = static_cast<long long>(B) * N;
+  const long long qbytes = rows * Hq * D * 2, kvbytes = rows * Hkv * D * 2;
+  if (overlaps(ws, ws_bytes, q, qbytes) || overlaps(ws, ws_bytes, o, qbytes) ||
+      overlaps(ws, ws_bytes, k, kvbytes) || overlaps(ws, ws_bytes, v, kvbytes))
+    return TM_ERR_INVALID_ARG;
+  return TM_OK;
+}
+
 int run(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv, int N, int D,
-        float scale, const trimix::Pattern& pat, void* stream) {
+        float scale, const trimix::Pattern& pat, void* ws, long long ws_bytes, void* stream) {
   trimix::LaunchArgs a;
   a.q = q; a.k = k; a.v = v; a.o = o;
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.N = N; a.D = D;
   a.scale = scale;
   a.pat = pat;
+  a.ws = ws;
+  a.ws_bytes = ws_bytes;
   a.stream = stream;
   return trimix::launch_attention(a);
 }
@@ -60,26 +77,67 @@ int run(const void* q, const void* k, const void* v, void* o, int B, int Hq, int
 
 extern "C" {
 
+TM_API int tm_causal_attn_fwd_ws(const void* q, const void* k, const void* v, void* o, int B,
+                                 int Hq, int Hkv, int N, int D, float scale, void* workspace,
+                                 long long workspace_bytes, void* stream) {
+  if (int rc = validate_common(q, k, v, o, B, Hq, Hkv, N, D, scale)) return rc;
+  if (int rc = validate_workspace(q, k, v, o, B, Hq, Hkv, N, D, workspace, workspace_bytes))
+    return rc;
+  return run(q, k, v, o, B, Hq, Hkv, N, D, scale, trimix::make_pattern(N, 1, 0, 1, 0), workspace,
+             workspace_bytes, stream);
+}
+
+TM_API int tm_triangle_attn_fwd_ws(const void* q, const void* k, const void* v, void* o, int B,
+                                   int Hq, int Hkv, int N, int D, float scale, int S, int W, int L,
+                                   void* workspace, long long workspace_bytes, void* stream) {
+  if (int rc = validate_common(q, k, v, o, B, Hq, Hkv, N, D, scale)) return rc;
+  if (int rc = validate_pattern(S, W, L)) return rc;
+  if (int rc = validate_workspace(q, k, v, o, B, Hq, Hkv, N, D, workspace, workspace_bytes))
+    return rc;
+  return run(q, k, v, o, B, Hq, Hkv, N, D, scale, trimix::make_pattern(N, 0, S, W, L), workspace,
+             workspace_bytes, stream);
+}
+
+TM_API int tm_trianglemix_attn_fwd_ws(const void* q, const void* k, const void* v, void* o, int B,
+                                      int Hq, int Hkv, int N, int D, float scale, int S, int W,
+                                      int L, int layer, int tri_start, void* workspace,
+                                      long long workspace_bytes, void* stream) {
+  if (layer < 0 || tri_start < 0) return TM_ERR_INVALID_ARG;
+  if (layer < tri_start)
+    return tm_causal_attn_fwd_ws(q, k, v, o, B, Hq, Hkv, N, D, scale, workspace, workspace_bytes,
+                                 stream);
+  return tm_triangle_attn_fwd_ws(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L, workspace,
+                                 workspace_bytes, stream);
+}
+
 TM_API int tm_causal_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int Hq,
                               int Hkv, int N, int D, float scale, void* stream) {
-  if (int rc = validate_common(q, k, v, o, B, Hq, Hkv, N, D, scale)) return rc;
-  return run(q, k, v, o, B, Hq, Hkv, N, D, scale, trimix::make_pattern(N, 1, 0, 1, 0), stream);
+  return tm_causal_attn_fwd_ws(q, k, v, o, B, Hq, Hkv, N, D, scale, nullptr, 0, stream);
 }
 
 TM_API int tm_triangle_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int Hq,
                                 int Hkv, int N, int D, float scale, int S, int W, int L,
                                 void* stream) {
-  if (int rc = validate_common(q, k, v, o, B, Hq, Hkv, N, D, scale)) return rc;
-  if (int rc = validate_pattern(S, W, L)) return rc;
-  return run(q, k, v, o, B, Hq, Hkv, N, D, scale, trimix::make_pattern(N, 0, S, W, L), stream);
+  return tm_triangle_attn_fwd_ws(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L, nullptr, 0, stream);
 }
 
 TM_API int tm_trianglemix_attn_fwd(const void* q, const void* k, const void* v, void* o, int B,
                                    int Hq, int Hkv, int N, int D, float scale, int S, int W, int L,
                                    int layer, int tri_start, void* stream) {
-  if (layer < 0 || tri_start < 0) return TM_ERR_INVALID_ARG;
-  if (layer < tri_start) return tm_causal_attn_fwd(q, k, v, o, B, Hq, Hkv, N, D, scale, stream);
-  return tm_triangle_attn_fwd(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L, stream);
+  return tm_trianglemix_attn_fwd_ws(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L, layer,
+                                    tri_start, nullptr, 0, stream);
+}
+
+TM_API int tm_attn_workspace_size(int B, int Hq, int Hkv, int N, int D, int causal, int S, int W,
+                                  int L, int num_ctas, long long* bytes) {
+  if (!bytes || B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0) return TM_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return TM_ERR_UNSUPPORTED;
+  if (!causal && validate_pattern(S, W, L)) return TM_ERR_INVALID_ARG;
+  if (static_cast<long long>((N + TM_BLOCK_M - 1) / TM_BLOCK_M) * B * Hkv * ((Hq / Hkv + 1) / 2) >
+      (1LL << 31) - 1)
+    return TM_ERR_INVALID_ARG;
+  return trimix::workspace_bytes(B, Hq, Hkv, N, D, trimix::make_pattern(N, causal, S, W, L),
+                                 num_ctas, bytes);
 }
 
 TM_API long long tm_triangle_kept_pairs(int N, int S, int W, int L) {
@@ -155,7 +213,7 @@ TM_API int tm_debug_mma_probe(const void* q, const void* k, const void* v, float
 }
 
 TM_API int tm_debug_schedule(int B, int Hq, int Hkv, int N, int causal, int S, int W, int L,
-                             int num_ctas, int* out, long long cap, long long* count) {
+                             int num_ctas, int split, int* out, long long cap, long long* count) {
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0 || num_ctas < 1 || cap < 0 || !count ||
       (cap > 0 && !out))
     return TM_ERR_INVALID_ARG;
@@ -164,7 +222,7 @@ TM_API int tm_debug_schedule(int B, int Hq, int Hkv, int N, int causal, int S, i
       (1LL << 31) - 1)
     return TM_ERR_INVALID_ARG;
   return trimix::debug_schedule(B, Hq, Hkv, N, trimix::make_pattern(N, causal, S, W, L), num_ctas,
-                                out, cap, count);
+                                split, out, cap, count);
 }
 
 TM_API int tm_get_device_status(void* stream) { return trimix::read_and_clear_device_status(stream); }

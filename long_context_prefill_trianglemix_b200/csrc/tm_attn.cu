@@ -85,6 +85,13 @@ static_assert(kPolyPairs >= 0 && kPolyPairs <= 32, "pairs per 32");
 // visited tile, used only to balance the persistent work split.
 constexpr long long kItemOverheadTiles = 3;
 constexpr uint64_t kDrainLimitNs = 100000000ull;
+// Cutting heavy items (split schedules): a piece costs at most this fraction
+// of a CTA's share, holds at least kMinPieceTiles tiles, an item is cut into
+// at most kMaxSplit pieces, and writing a partial costs about one tile.
+constexpr double kSplitShare = 0.5;
+constexpr int kMinPieceTiles = 8;
+constexpr int kMaxSplit = 16;
+constexpr long long kSplitOverheadTiles = 1;
 
 // Where a wait gave up (recorded with the timeout, for diagnosis).
 enum WaitSite : int {
@@ -126,17 +133,35 @@ struct AttnParams {
   Pattern pat;
   float sl2;  // softmax scale * log2(e)
   // Items run q-block major (longest q-blocks first), the (batch, kv head,
-  // pair) units inside. The first n_big items (the n_hqb heaviest q-blocks, the
-  // last-L blocks of the triangle) are dealt round-robin: CTA c takes c,
-  // c + grid, ... Every other item is dealt in strided rounds, so that the CTAs
-  // running at the same time work on neighbouring q-blocks of every kv head and
-  // each K/V tile is read from DRAM about once per round. The first n_a CTAs
-  // hold one big item more than the rest and join the rounds n_skip rounds
-  // late. Normal item j of CTA c (j counted from 0):
+  // pair) units inside. The n_hqb heaviest q-blocks (the last-L blocks of the
+  // triangle) give n_hunits = n_hqb * units heavy items; those of the first
+  // n_sqb q-blocks are each cut into nsplit pieces of their tile list. The
+  // n_big big pieces (n_sbig = n_sqb * units * nsplit pieces of cut items,
+  // then the other heavy items whole) are dealt round-robin: CTA c takes c,
+  // c + grid, ... Every other item is dealt in
+  // strided rounds, so that the CTAs running at the same time work on
+  // neighbouring q-blocks of every kv head and each K/V tile is read from DRAM
+  // about once per round. The first n_a CTAs hold one piece more than the rest
+  // and join the rounds n_skip rounds late. Normal item j of CTA c (j counted
+  // from 0, item index n_hunits + that):
   //   c >= n_a and j < n_skip:  (c - n_a) + j * (grid - n_a)
   //   otherwise:                 n_skip * (grid - n_a) + (j - s_c) * grid + c,
   //                              s_c = n_skip if c >= n_a else 0
-  int n_hqb, n_big, n_a, n_skip;
+  int n_hqb, n_hunits, n_sqb, n_sbig, n_big, n_a, n_skip;
+  // With an odd group size one pair per kv head holds a single Q tile. The
+  // pair of an item is rotated by pair_rot per q-block slot (pair digit + qi *
+  // pair_rot, mod npairs), chosen so that the pair a CTA gets changes through
+  // all npairs values along its stride and every CTA gets its share of the
+  // cheap single-tile items (0 for even group sizes). The rotation permutes
+  // the pairs inside each (kv head, q-block) group, whose items stay adjacent.
+  int pair_rot;
+  // Split pieces (nsplit > 1): each writes its unnormalised partial (O, running
+  // max m, sum l) of every 32-row warp slice to ws_rec and counts itself in
+  // ws_cnt (one counter per cut item, Q tile and warp, zero at launch); the
+  // piece that arrives last merges all partials in split order.
+  int nsplit;
+  float* ws_rec;
+  int* ws_cnt;
 };
 
 __host__ __device__ __forceinline__ int big_count(const AttnParams& p, int c, int g) {
@@ -154,7 +179,7 @@ __host__ __device__ __forceinline__ long long normal_index(const AttnParams& p, 
 }
 
 __host__ __device__ __forceinline__ int work_count(const AttnParams& p, int c, int g) {
-  const long long n_norm = static_cast<long long>(p.nqb) * p.units - p.n_big;
+  const long long n_norm = static_cast<long long>(p.nqb) * p.units - p.n_hunits;
   // largest j with normal_index(j) < n_norm, + 1 (monotone in j)
   int lo = 0, hi = static_cast<int>(n_norm) + 1;
   while (lo < hi) {
@@ -169,21 +194,57 @@ __host__ __device__ __forceinline__ int work_item(const AttnParams& p, int c, in
   return k < nb ? c + k * g : p.n_big + static_cast<int>(normal_index(p, c, g, k - nb));
 }
 
+// One unit of work: Q tiles h0 (and h0 + 1 if v1) of q-block qb, kv head g of
+// batch b, over tiles [t0, min(t1, count)) of the q-block's tile list. split
+// >= 0 marks a piece of a heavy item (hunit: its index among the heavy items).
 struct Item {
   int b, g, qb, h0, v1;
+  int t0, t1, split, hunit;
 };
+
+constexpr int kAllTiles = 0x7fffffff;
 
 __host__ __device__ __forceinline__ Item decode_item(const AttnParams& p, int item) {
   Item it;
   const int qi = item / p.units;
   const int u = item - qi * p.units;
   it.qb = p.nqb - 1 - qi;  // longest q-blocks first
-  const int pr = u % p.npairs;
+  // unit digits, fastest first: pair, kv head, batch. The pairs of one kv head
+  // and q-block are consecutive items, which the strided rounds hand to
+  // neighbouring CTAs: they walk the same tile list in lockstep, so each K/V
+  // tile is fetched from DRAM once for all of them.
+  const int pr = (u % p.npairs + static_cast<int>(static_cast<long long>(qi) * p.pair_rot % p.npairs)) %
+                 p.npairs;
   const int gb = u / p.npairs;
   it.g = gb % p.Hkv;
   it.b = gb / p.Hkv;
   it.h0 = it.g * p.G + 2 * pr;
   it.v1 = (2 * pr + 1 < p.G) ? 1 : 0;
+  it.t0 = 0;
+  it.t1 = kAllTiles;
+  it.split = -1;
+  it.hunit = -1;
+  return it;
+}
+
+// Big piece bi < n_sbig: cut q-block slot qi, then split s, then unit u (so
+// CTAs running at the same time read the same tile range of a kv head); the
+// rest are whole heavy items in item order.
+__host__ __device__ __forceinline__ Item decode_piece(const AttnParams& p, int bi) {
+  if (bi >= p.n_sbig) return decode_item(p, p.n_sqb * p.units + (bi - p.n_sbig));
+  const int per_q = p.units * p.nsplit;
+  const int qi = bi / per_q;
+  const int rem = bi - qi * per_q;
+  const int s = rem / p.units;
+  const int u = rem - s * p.units;
+  Item it = decode_item(p, qi * p.units + u);
+  if (p.nsplit > 1) {
+    const int T = block_tiles(p.pat, it.qb, BM, BN).count();
+    it.t0 = static_cast<int>(static_cast<long long>(T) * s / p.nsplit);
+    it.t1 = static_cast<int>(static_cast<long long>(T) * (s + 1) / p.nsplit);
+    it.split = s;
+    it.hunit = qi * p.units + u;
+  }
   return it;
 }
 
@@ -197,6 +258,7 @@ struct WorkCursor {
   int j, phase_end;                 // normal position; where the current stride ends
   int pr, kvh, b, qi;               // digits of the next normal item
   int d_pr, d_kvh, d_b, d_qi;       // digits of the current stride
+  int rot, d_rot;                   // qi * pair_rot and d_qi * pair_rot, mod npairs
   __host__ __device__ __forceinline__ void set_item(const AttnParams& p, long long item) {
     qi = static_cast<int>(item / p.units);
     const int u = static_cast<int>(item - static_cast<long long>(qi) * p.units);
@@ -204,6 +266,7 @@ struct WorkCursor {
     const int gb = u / p.npairs;
     kvh = gb % p.Hkv;
     b = gb / p.Hkv;
+    rot = static_cast<int>(static_cast<long long>(qi) * p.pair_rot % p.npairs);
   }
   __host__ __device__ __forceinline__ void set_stride(const AttnParams& p, int stride) {
     d_qi = stride / p.units;
@@ -212,9 +275,10 @@ struct WorkCursor {
     const int gb = u / p.npairs;
     d_kvh = gb % p.Hkv;
     d_b = gb / p.Hkv;
+    d_rot = static_cast<int>(static_cast<long long>(d_qi) * p.pair_rot % p.npairs);
   }
   __host__ __device__ __forceinline__ void enter_phase(const AttnParams& p) {
-    set_item(p, p.n_big + normal_index(p, c, g, j));
+    set_item(p, p.n_hunits + normal_index(p, c, g, j));
     const bool late = c >= p.n_a && j < p.n_skip;
     set_stride(p, late ? g - p.n_a : g);
     phase_end = late ? p.n_skip : 0x7fffffff;
@@ -234,14 +298,20 @@ struct WorkCursor {
   __host__ __device__ __forceinline__ Item next(const AttnParams& p) {
     Item it;
     if (k < nb) {
-      it = decode_item(p, big_next);
+      it = decode_piece(p, big_next);
       big_next += g;
     } else {
+      it.t0 = 0;
+      it.t1 = kAllTiles;
+      it.split = -1;
+      it.hunit = -1;
       it.qb = p.nqb - 1 - qi;
       it.g = kvh;
       it.b = b;
-      it.h0 = kvh * p.G + 2 * pr;
-      it.v1 = (2 * pr + 1 < p.G) ? 1 : 0;
+      int pe = pr + rot;
+      if (pe >= p.npairs) pe -= p.npairs;
+      it.h0 = kvh * p.G + 2 * pe;
+      it.v1 = (2 * pe + 1 < p.G) ? 1 : 0;
       ++j;
       if (j == phase_end) {
         enter_phase(p);
@@ -256,6 +326,9 @@ struct WorkCursor {
         carry = 0;
         if (b >= p.B) { b -= p.B; carry = 1; }
         qi += d_qi + carry;
+        rot += d_rot + (carry ? p.pair_rot : 0);  // < 3 npairs
+        if (rot >= p.npairs) rot -= p.npairs;
+        if (rot >= p.npairs) rot -= p.npairs;
       }
     }
     ++k;
@@ -367,8 +440,8 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, Bars<Cfg<D>::
                     it.h0 + 1, it.qb * BM, it.b);
     }
     ++it_cnt;
-    const int T = bt.count();
-    for (int t = 0; ok && t < T; ++t) {
+    const int t_end = imin(bt.count(), it.t1);
+    for (int t = it.t0; ok && t < t_end; ++t) {
       const int kb = bt.kb(t);
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
@@ -419,7 +492,7 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStag
   cur.init(p, blockIdx.x, gridDim.x);
   while (ok && !cur.done()) {
     const Item it = cur.next(p);
-    const int T = block_tiles(p.pat, it.qb, BM, BN).count();
+    const int T = imin(block_tiles(p.pat, it.qb, BM, BN).count(), it.t1) - it.t0;
     const bool v1 = it.v1 != 0;
     TM_WAIT(&bars->q_full, it_cnt & 1u, kSiteQFull);
     ++it_cnt;
@@ -486,6 +559,77 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStag
   drain_wait(&bars->mma_done, 0);
 }
 
+// Split pieces of a heavy item: this warp's 32 rows of the piece's partial
+// (unnormalised O, running max m, sum l, all in the log2 domain of m) go to its
+// record; record layout: O as float4[D/4][128] (a warp's 16-byte stores cover
+// 512 contiguous bytes), then m[128], l[128]. The warp then counts itself in
+// its counter; the warp that arrives last (no waiting: the others leave)
+// merges all nsplit partials in split order, so the result does not depend on
+// which piece finished last, and returns true with orr / l_run replaced by the
+// merged O and l. No thread ever waits on another CTA.
+template <int D>
+__device__ __forceinline__ bool merge_split(const AttnParams& p, const Item& it, int wg, int wq,
+                                            int lane, uint32_t (&orr)[D / 32][32], float m_run,
+                                            float& l_run) {
+  constexpr int kRecFloats = 128 * D + 256;
+  const int r = wq * 32 + lane;
+  float* recs = p.ws_rec + static_cast<size_t>(it.hunit) * p.nsplit * 2 * kRecFloats;
+  {
+    float* rec = recs + static_cast<size_t>(it.split * 2 + wg) * kRecFloats;
+    float4* ro = reinterpret_cast<float4*>(rec);
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c)
+#pragma unroll
+      for (int x = 0; x < 8; ++x)
+        __stcg(ro + (c * 8 + x) * 128 + r,
+               make_float4(__uint_as_float(orr[c][4 * x]), __uint_as_float(orr[c][4 * x + 1]),
+                           __uint_as_float(orr[c][4 * x + 2]), __uint_as_float(orr[c][4 * x + 3])));
+    __stcg(rec + 128 * D + r, m_run);
+    __stcg(rec + 128 * D + 128 + r, l_run);
+  }
+  __threadfence();
+  __syncwarp();
+  int last = 0;
+  if (lane == 0) {
+    last = atomicAdd(p.ws_cnt + (it.hunit * 2 + wg) * 4 + wq, 1) == p.nsplit - 1;
+    __threadfence();
+  }
+  if (!__shfl_sync(0xffffffffu, last, 0)) return false;
+  float M = -INFINITY;
+  for (int sp = 0; sp < p.nsplit; ++sp)
+    M = fmaxf(M, __ldcg(recs + static_cast<size_t>(sp * 2 + wg) * kRecFloats + 128 * D + r));
+  float acc[D / 32][32];
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c)
+#pragma unroll
+    for (int x = 0; x < 32; ++x) acc[c][x] = 0.f;
+  float l_sum = 0.f;
+#pragma unroll 1
+  for (int sp = 0; sp < p.nsplit; ++sp) {
+    const float* rec = recs + static_cast<size_t>(sp * 2 + wg) * kRecFloats;
+    const float ms = __ldcg(rec + 128 * D + r);
+    const float w = ms == -INFINITY ? 0.f : ex2(ms - M);
+    l_sum = fmaf(w, __ldcg(rec + 128 * D + 128 + r), l_sum);
+    const float4* ro = reinterpret_cast<const float4*>(rec);
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c)
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        const float4 v = __ldcg(ro + (c * 8 + x) * 128 + r);
+        acc[c][4 * x] = fmaf(w, v.x, acc[c][4 * x]);
+        acc[c][4 * x + 1] = fmaf(w, v.y, acc[c][4 * x + 1]);
+        acc[c][4 * x + 2] = fmaf(w, v.z, acc[c][4 * x + 2]);
+        acc[c][4 * x + 3] = fmaf(w, v.w, acc[c][4 * x + 3]);
+      }
+  }
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c)
+#pragma unroll
+    for (int x = 0; x < 32; ++x) orr[c][x] = __float_as_uint(acc[c][x]);
+  l_run = l_sum;
+  return true;
+}
+
 template <int D>
 __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::kStages>* bars,
                                              uint8_t* smem, const CUtensorMap* to, int wg, int wq,
@@ -504,7 +648,7 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
     const Item it = cur.next(p);
     if (wg == 1 && !it.v1) continue;
     const BlockTiles bt = block_tiles(pat, it.qb, BM, BN);
-    const int T = bt.count();
+    const int T = imin(bt.count(), it.t1) - it.t0;
     const int i = it.qb * BM + r;  // query row of this thread
     // kept keys of row i: [0, sink_hi) U [band_lo, hi)
     const int hi = imin(i, pat.N - 1) + 1;
@@ -513,7 +657,7 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
     const int band_lo = full_row ? hi : imax(0, i - pat.W + 1);
     float m_run = -INFINITY, l_run = 0.f;
     for (int t = 0; t < T; ++t) {
-      const int kb = bt.kb(t);
+      const int kb = bt.kb(it.t0 + t);
       const bool need_mask = tile_needs_mask(pat, it.qb, kb, BM, BN) != 0;
       bool ok = wait_bar(&bars->s_full[wg], s_cnt & 1u, abort_flag, kSiteSFull);
       ++s_cnt;
@@ -619,6 +763,7 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
     for (int c = 1; c < D / 32; ++c) reg_fence(orr[c]);
     tc_fence_before();
     mbar_arrive(&bars->o_empty[wg]);
+    if (it.split >= 0 && !merge_split<D>(p, it, wg, wq, lane, orr, m_run, l_run)) continue;
     const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
     const uint32_t slot = smem_addr(smem + Cfg<D>::kStageOff) + (wg * 4 + wq) * Cfg<D>::kStageSlotBytes;
     const uint32_t row_addr = slot + lane * 128;
@@ -897,18 +1042,23 @@ int encode_bnhd(CUtensorMap* m, const void* base, int B, int N, int H, int D, in
   return r == CUDA_SUCCESS ? TM_OK : TM_ERR_CUDA;
 }
 
-// Fills the geometry and the persistent work split of *p; returns the grid size.
-int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ctas, AttnParams* p) {
+// Fills the geometry and the persistent work split of *p; returns the grid
+// size. split: heavy items may be cut into pieces (the caller has workspace).
+int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ctas, bool split,
+                   AttnParams* p) {
   p->B = B; p->Hq = Hq; p->Hkv = Hkv; p->N = N;
   p->G = Hq / Hkv;
   p->npairs = (p->G + 1) / 2;
   p->nqb = (N + BM - 1) / BM;
   p->units = B * Hkv * p->npairs;
   p->pat = pat;
+  p->ws_rec = nullptr;
+  p->ws_cnt = nullptr;
+  p->pair_rot = 0;
   // Persistent grid. Item cost = (visited tiles + fixed per-item overhead,
   // about the pipeline fill/drain and epilogue) x Q tiles of the item; it is
-  // used to find the heavy q-blocks and how many rounds the CTAs holding an
-  // extra heavy item sit out.
+  // used to find the heavy q-blocks, how finely to cut them, and how many
+  // rounds the CTAs holding an extra heavy piece sit out.
   const long long n_items = static_cast<long long>(p->nqb) * p->units;
   const int grid = static_cast<int>(std::min<long long>(std::min(max_ctas, kMaxCtas), n_items));
   std::vector<long long> qcost(p->nqb);
@@ -926,15 +1076,50 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
          static_cast<long long>(n_hqb + 1) * p->units <= 8LL * grid)
     ++n_hqb;
   p->n_hqb = n_hqb;
-  p->n_big = n_hqb * p->units;
+  p->n_hunits = n_hqb * p->units;
+  // Cut the heavy q-blocks whose items cost more than kSplitShare of a CTA's
+  // share into ns pieces (ns from the heaviest, so its pieces fit that share),
+  // each of at least kMinPieceTiles tiles, at most 8 big pieces per CTA.
+  int ns = 1, n_sqb = 0;
+  if (split && n_hqb > 0) {
+    const double heavy = static_cast<double>(qcost[p->nqb - 1] * item_q);
+    ns = static_cast<int>(std::ceil(heavy / (kSplitShare * target)));
+    ns = std::min(ns, std::max(1, block_tiles(p->pat, p->nqb - 1, BM, BN).count() / kMinPieceTiles));
+    ns = std::min(ns, kMaxSplit);
+    while (n_sqb < n_hqb && qcost[p->nqb - 1 - n_sqb] * item_q > kSplitShare * target &&
+           block_tiles(p->pat, p->nqb - 1 - n_sqb, BM, BN).count() >= ns * kMinPieceTiles)
+      ++n_sqb;
+    ns = std::min(ns, std::max(1, static_cast<int>(
+                              (8LL * grid - (n_hqb - n_sqb) * static_cast<long long>(p->units)) /
+                              std::max(1LL, static_cast<long long>(n_sqb) * p->units))));
+    if (ns <= 1 || n_sqb == 0) { ns = 1; n_sqb = 0; }
+  }
+  p->nsplit = ns;
+  p->n_sqb = n_sqb;
+  p->n_sbig = n_sqb * p->units * ns;
+  p->n_big = p->n_sbig + (n_hqb - n_sqb) * p->units;
+  if (p->G % 2 == 1 && p->npairs > 1) {
+    // per stride of grid items the pair digit advances by d_pr (plus carries)
+    // and the q-block slot by d_qi; take the first rotation that makes the
+    // advance coprime with npairs
+    const int d_qi = grid / p->units;
+    const int d_pr = (grid % p->units) % p->npairs;
+    for (int r = 0; r < p->npairs; ++r) {
+      int a = (d_pr + d_qi * r) % p->npairs, b = p->npairs;
+      while (b) { const int t = a % b; a = b; b = t; }
+      if (a == 1) { p->pair_rot = r; break; }
+    }
+  }
   p->n_a = 0;
   p->n_skip = 0;
-  const long long n_norm = n_items - p->n_big;
+  const long long n_norm = n_items - p->n_hunits;
   if (p->n_big % grid != 0 && n_norm > 0) {
-    // CTAs [0, n_a) hold one big item more; they sit out the rounds that the
+    // CTAs [0, n_a) hold one big piece more; they sit out the rounds that the
     // others spend on an equal cost of normal items
     double big_cost = 0, norm_cost = 0;
-    for (int q = 0; q < n_hqb; ++q) big_cost += qcost[p->nqb - 1 - q];
+    for (int q = 0; q < n_hqb; ++q)
+      big_cost += qcost[p->nqb - 1 - q] +
+                  (q < n_sqb ? ns * kSplitOverheadTiles + (ns - 1) * kItemOverheadTiles : 0);
     big_cost = big_cost * B * Hq / p->n_big;
     for (int qb = 0; qb < p->nqb - n_hqb; ++qb) norm_cost += qcost[qb];
     norm_cost = norm_cost * B * Hq / n_norm;
@@ -944,6 +1129,22 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
     p->n_skip = static_cast<int>(std::min<long long>(max_rounds, static_cast<long long>(rounds + 0.5)));
   }
   return grid;
+}
+
+// Workspace of a split schedule: the arrival counters (one int per cut item,
+// Q tile and warp, padded to 256 bytes), then one partial record per cut
+// item, piece and Q tile. 0 when nothing is split.
+struct WsLayout {
+  long long cnt_bytes, total;
+};
+WsLayout ws_layout(const AttnParams& p, int D) {
+  WsLayout w{0, 0};
+  if (p.nsplit <= 1) return w;
+  const long long n_cut = static_cast<long long>(p.n_sqb) * p.units;  // items that are cut
+  w.cnt_bytes = (n_cut * 8 * 4 + 255) / 256 * 256;
+  const long long rec_bytes = (128LL * D + 256) * 4;
+  w.total = w.cnt_bytes + n_cut * p.nsplit * 2 * rec_bytes;
+  return w;
 }
 
 template <int D>
@@ -971,9 +1172,16 @@ int launch_attention_d(const LaunchArgs& a, DeviceInfo* di) {
     return TM_ERR_CUDA;
 
   AttnParams p;
+  const int grid = build_schedule(a.B, a.Hq, a.Hkv, a.N, a.pat, di->sms, a.ws != nullptr, &p);
   p.sl2 = a.scale * 1.4426950408889634f;
-
-  const int grid = build_schedule(a.B, a.Hq, a.Hkv, a.N, a.pat, di->sms, &p);
+  const WsLayout w = ws_layout(p, D);
+  if (w.total > 0) {
+    if (a.ws_bytes < w.total) return TM_ERR_INVALID_ARG;
+    p.ws_cnt = static_cast<int*>(a.ws);
+    p.ws_rec = reinterpret_cast<float*>(static_cast<uint8_t*>(a.ws) + w.cnt_bytes);
+    if (cudaMemsetAsync(a.ws, 0, w.cnt_bytes, static_cast<cudaStream_t>(a.stream)) != cudaSuccess)
+      return TM_ERR_CUDA;
+  }
   attn_kernel<D><<<grid, kThreads, Cfg<D>::kSmemBytes, static_cast<cudaStream_t>(a.stream)>>>(
       tq, tk, tv, to, p);
   return cudaGetLastError() == cudaSuccess ? TM_OK : TM_ERR_CUDA;
@@ -989,10 +1197,24 @@ int launch_attention(const LaunchArgs& a) {
   return TM_ERR_UNSUPPORTED;
 }
 
-int debug_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ctas, int* out,
-                   long long cap, long long* count) {
+int workspace_bytes(int B, int Hq, int Hkv, int N, int D, const Pattern& pat, int num_ctas,
+                    long long* bytes) {
+  if (num_ctas <= 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&num_ctas, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return TM_ERR_CUDA;
+  }
   AttnParams p;
-  const int grid = build_schedule(B, Hq, Hkv, N, pat, max_ctas, &p);
+  build_schedule(B, Hq, Hkv, N, pat, num_ctas, true, &p);
+  *bytes = ws_layout(p, D).total;
+  return TM_OK;
+}
+
+int debug_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ctas, int split,
+                   int* out, long long cap, long long* count) {
+  AttnParams p;
+  const int grid = build_schedule(B, Hq, Hkv, N, pat, max_ctas, split != 0, &p);
   long long n = 0;
   for (int c = 0; c < grid; ++c) {
     WorkCursor cur;
@@ -1001,12 +1223,16 @@ int debug_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
     for (int k = 0; !cur.done(); ++k, ++n) {
       const Item it = cur.next(p);  // what the kernel's roles see
       const int item = work_item(p, c, grid, k);
-      const Item ref = decode_item(p, item);
-      if (it.qb != ref.qb || it.b != ref.b || it.g != ref.g || it.h0 != ref.h0 || it.v1 != ref.v1)
+      const Item ref = item < p.n_big ? decode_piece(p, item)
+                                      : decode_item(p, item - p.n_big + p.n_hunits);
+      if (it.qb != ref.qb || it.b != ref.b || it.g != ref.g || it.h0 != ref.h0 || it.v1 != ref.v1 ||
+          it.t0 != ref.t0 || it.t1 != ref.t1 || it.split != ref.split || it.hunit != ref.hunit)
         return TM_ERR_INVALID_ARG;  // the cursor and the direct decode disagree
       if (n >= cap) continue;
-      int* r = out + 5 * n;
+      const int T = block_tiles(p.pat, it.qb, BM, BN).count();
+      int* r = out + 7 * n;
       r[0] = c; r[1] = item; r[2] = it.qb; r[3] = it.b * Hq + it.h0; r[4] = 1 + it.v1;
+      r[5] = it.t0; r[6] = std::min(T, it.t1);
     }
   }
   *count = n;

@@ -19,6 +19,8 @@ struct LaunchArgs {
   int B, Hq, Hkv, N, D;
   float scale;
   Pattern pat;
+  void* ws;           // split workspace (device), or nullptr: no item is split
+  long long ws_bytes;
   void* stream;
 };
 
@@ -28,7 +30,11 @@ int launch_dump_tiles(const Pattern& p, int* out_dev, long long cap, void* strea
 int launch_mma_probe(const void* q, const void* k, const void* v, float* s_out, float* o_out,
                      int D, void* stream);
 int read_and_clear_device_status(void* stream);
-int debug_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ctas, int* out,
-                   long long cap, long long* count);
+int debug_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ctas, int split,
+                   int* out, long long cap, long long* count);
+// Workspace bytes the split schedule needs on num_ctas CTAs (<= 0: the
+// current device's SM count); 0 if no item is split.
+int workspace_bytes(int B, int Hq, int Hkv, int N, int D, const Pattern& pat, int num_ctas,
+                    long long* bytes);
 
 }  // namespace trimix

@@ -126,7 +126,7 @@ class Workload:
         return layer if self.seed_is_layer else 0
 
 
-# The five workloads: shapes of Llama-3-8B (32 q heads, 8 kv heads, head dim
+# The workloads: shapes of Llama-3-8B (32 q heads, 8 kv heads, head dim
 # 128, 32 layers) and Qwen2.5-7B (28 q heads, 4 kv heads, 28 layers) with the
 # layer splits the blog post reports (12 dense layers for Llama-3, 20 for
 # Qwen2.5; section 性能) and triangle parameters S/W/L chosen per workload.
@@ -144,6 +144,14 @@ WORKLOADS = {
     "qwen2.5-7b-128k-28layer": Workload("qwen2.5-7b-128k-28layer", B=1, Hq=28, Hkv=4,
                                         N=131072, D=128, S=64, W=1024, L=128, layers=28,
                                         tri_start=20, recipe="headscale"),
+    # One GPU's share of the same layers under tensor parallelism (heads split
+    # over 8 and 4 GPUs): few heads per launch, so each last-L item is a large
+    # fraction of the launch and is cut into pieces when a workspace is given.
+    "llama3-8b-128k-tp8": Workload("llama3-8b-128k-tp8", B=1, Hq=4, Hkv=1, N=131072, D=128,
+                                   S=64, W=2048, L=256, layers=2, tri_start=1),
+    "qwen2.5-7b-128k-tp4": Workload("qwen2.5-7b-128k-tp4", B=1, Hq=7, Hkv=1, N=131072, D=128,
+                                    S=64, W=1024, L=128, layers=28, tri_start=20,
+                                    recipe="headscale"),
 }
 
 

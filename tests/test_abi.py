@@ -134,3 +134,31 @@ def test_kept_pairs_and_tiles():
         assert tm.tm_triangle_kept_pairs(N, S, W, L) == oracle.kept_pairs(N, False, S, W, L)
     assert tm.tm_kept_tiles(131072, True, 0, 1, 0) == 1024 * 1025 // 2
     assert tm.tm_triangle_kept_pairs(10, 0, 0, 0) == -1
+
+
+WS_ARGS = (FAKE, FAKE, FAKE, FAKE + 0x100000, 1, 4, 4, 64, 64, 0.1)
+
+
+@pytest.mark.parametrize("ws,nbytes", [(0, 256), (FAKE + 0x200008, 256), (FAKE + 0x200000, -1),
+                                       (FAKE + 0x100, 4096), (FAKE + 0x100000 - 64, 4096)])
+def test_workspace_validation(ws, nbytes):
+    L = tm.lib()
+    assert L.tm_triangle_attn_fwd_ws(*WS_ARGS, 4, 8, 2, ws, nbytes, None) == tm.TM_ERR_INVALID_ARG
+    assert L.tm_causal_attn_fwd_ws(*WS_ARGS, ws, nbytes, None) == tm.TM_ERR_INVALID_ARG
+    assert L.tm_trianglemix_attn_fwd_ws(*WS_ARGS, 4, 8, 2, 3, 1, ws, nbytes,
+                                        None) == tm.TM_ERR_INVALID_ARG
+
+
+def test_workspace_size_arguments():
+    n = ctypes.c_longlong(-1)
+    L = tm.lib()
+    assert L.tm_attn_workspace_size(1, 4, 3, 4096, 128, 0, 0, 1, 0, 148, ctypes.byref(n)) == \
+        tm.TM_ERR_INVALID_ARG
+    assert L.tm_attn_workspace_size(1, 4, 1, 4096, 96, 0, 0, 1, 0, 148, ctypes.byref(n)) == \
+        tm.TM_ERR_UNSUPPORTED
+    assert L.tm_attn_workspace_size(1, 4, 1, 4096, 128, 0, 0, 0, 0, 148, ctypes.byref(n)) == \
+        tm.TM_ERR_INVALID_ARG
+    assert L.tm_attn_workspace_size(1, 4, 1, 4096, 128, 0, 0, 1, 0, 148, None) == \
+        tm.TM_ERR_INVALID_ARG
+    assert L.tm_attn_workspace_size(1, 4, 1, 4096, 128, 0, 16, 64, 64, 148, ctypes.byref(n)) == 0
+    assert n.value >= 0

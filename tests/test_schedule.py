@@ -1,6 +1,8 @@
 """The persistent work split (host export of the same code the launch uses):
 every (q-block, q-head pair) item is processed exactly once, the longest
-items come first in each CTA, and the per-CTA cost is balanced."""
+items come first in each CTA, and the per-CTA cost is balanced. With a
+workspace the heavy items are cut into pieces whose tile ranges cover each
+item's tile list exactly once."""
 import numpy as np
 import pytest
 
@@ -32,7 +34,8 @@ def test_every_item_exactly_once(B, Hq, Hkv, N, causal, S, W, L):
     assert sorted(rec[:, 1].tolist()) == list(range(n_items))
     # every (batch, q head, q-block) tile appears once
     tiles = set()
-    for c, item, qb, h0, nv in rec:
+    for c, item, qb, h0, nv, t0, t1 in rec:
+        assert t0 == 0
         for h in range(h0, h0 + nv):
             assert (qb, h) not in tiles
             tiles.add((qb, h))
@@ -48,7 +51,7 @@ def test_triangle_split_is_balanced(N, S, W, L):
     tiles = tm.tm_tile_list(N, False, S, W, L)
     per_qb = np.bincount(tiles[:, 0], minlength=(N + 127) // 128)
     cost = np.zeros(148)
-    for c, item, qb, h0, nv in rec:
+    for c, item, qb, h0, nv, t0, t1 in rec:
         cost[c] += (per_qb[qb] + 3) * nv
     # within one normal item of the mean
     normal = (per_qb[:-3].max() + 3) * 2
@@ -78,3 +81,92 @@ def test_concurrent_items_share_kv_tiles(N, causal, W, L):
         it = rec[rec[:, 0] == c][:, 1]
         d = np.diff(it)
         assert (d > 0).all() and (d >= 100).all(), (c, it[:6])
+
+
+SPLIT_CASES = [(1, 4, 1, 131072, False, 64, 2048, 256), (1, 4, 1, 131072, False, 64, 512, 256),
+               (1, 8, 2, 65536, False, 64, 1024, 128), (1, 32, 8, 131072, False, 64, 512, 256),
+               (1, 4, 1, 131072, True, 0, 1, 0), (1, 2, 1, 32768, True, 0, 1, 0),
+               (1, 4, 4, 512, False, 16, 64, 64), (2, 6, 2, 1000, False, 3, 100, 300),
+               (1, 28, 4, 131072, False, 64, 1024, 128), (1, 7, 1, 65536, False, 64, 1024, 200)]
+
+
+def cta_costs(rec, per_qb, n_ctas=148, overhead=3, split_overhead=1):
+    cost = np.zeros(n_ctas)
+    for c, item, qb, h0, nv, t0, t1 in rec:
+        piece = (t1 - t0) + overhead + (split_overhead if t1 - t0 < per_qb[qb] else 0)
+        cost[c] += piece * nv
+    return cost
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,causal,S,W,L", SPLIT_CASES)
+def test_split_pieces_cover_each_item_once(B, Hq, Hkv, N, causal, S, W, L):
+    rec = tm.tm_debug_schedule(B, Hq, Hkv, N, causal, S, W, L, 148, split=True)
+    tiles = tm.tm_tile_list(N, causal, S, W, L)
+    per_qb = np.bincount(tiles[:, 0], minlength=(N + 127) // 128)
+    seen = {}
+    for c, item, qb, h0, nv, t0, t1 in rec:
+        assert 0 <= t0 < t1 <= per_qb[qb]
+        for h in range(h0, h0 + nv):
+            seen.setdefault((qb, h), []).append((t0, t1))
+    nqb = (N + 127) // 128
+    assert len(seen) == nqb * B * Hq
+    for (qb, h), ranges in seen.items():
+        ranges.sort()
+        assert ranges[0][0] == 0 and ranges[-1][1] == per_qb[qb], (qb, h, ranges)
+        for (a0, a1), (b0, b1) in zip(ranges, ranges[1:]):
+            assert a1 == b0, (qb, h, ranges)   # contiguous, no overlap
+    # the item ids are a permutation
+    assert sorted(rec[:, 1].tolist()) == list(range(len(rec)))
+    # pieces of one heavy item run on different CTAs, all before normal work
+    pieces = rec[(rec[:, 6] - rec[:, 5]) < per_qb[rec[:, 2]]]
+    for key in {(int(q), int(h)) for _, _, q, h, _, _, _ in pieces}:
+        ctas = pieces[(pieces[:, 2] == key[0]) & (pieces[:, 3] == key[1])][:, 0]
+        assert len(set(ctas.tolist())) == len(ctas)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,causal,S,W,L", [c for c in SPLIT_CASES if c[3] >= 32768])
+def test_split_balances_small_head_counts(B, Hq, Hkv, N, causal, S, W, L):
+    tiles = tm.tm_tile_list(N, causal, S, W, L)
+    per_qb = np.bincount(tiles[:, 0], minlength=(N + 127) // 128)
+    whole = cta_costs(tm.tm_debug_schedule(B, Hq, Hkv, N, causal, S, W, L, 148), per_qb)
+    split = cta_costs(tm.tm_debug_schedule(B, Hq, Hkv, N, causal, S, W, L, 148, split=True), per_qb)
+    # never worse than the unsplit schedule, and within about a fifth of the mean
+    assert split.max() <= whole.max() * 1.01
+    assert split.max() <= 1.2 * split.mean() or split.max() <= whole.max() * 0.5 + split.mean(), (
+        split.max(), split.mean(), whole.max())
+
+
+def test_split_needed_only_when_an_item_exceeds_its_share():
+    # Llama-3-8B at 128K with all 32 q heads: the last-L items fit in a CTA's share
+    assert tm.tm_attn_workspace_size(1, 32, 8, 131072, 128, False, 64, 2048, 256, 148) == 0
+    # a tensor-parallel shard (4 q heads, 1 kv head) has to cut them
+    n = tm.tm_attn_workspace_size(1, 4, 1, 131072, 128, False, 64, 2048, 256, 148)
+    assert n > 0
+    rec = tm.tm_debug_schedule(1, 4, 1, 131072, False, 64, 2048, 256, 148, split=True)
+    per_qb = np.bincount(tm.tm_tile_list(131072, False, 64, 2048, 256)[:, 0])
+    n_pieces = int(((rec[:, 6] - rec[:, 5]) < per_qb[rec[:, 2]]).sum())
+    ns = n_pieces // (2 * 2)          # 2 heavy q-blocks x 2 head pairs
+    cnt_bytes = -(-2 * 2 * 8 * 4 // 256) * 256
+    assert n == cnt_bytes + 2 * 2 * ns * 2 * (128 * 128 + 256) * 4
+    # D = 64 records are half the size
+    n64 = tm.tm_attn_workspace_size(1, 4, 1, 131072, 64, False, 64, 2048, 256, 148)
+    assert n64 == cnt_bytes + 2 * 2 * ns * 2 * (128 * 64 + 256) * 4
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,causal,W,L", [(1, 32, 8, 131072, False, 2048, 256),
+                                                   (1, 32, 8, 32768, True, 1, 0),
+                                                   (1, 28, 4, 131072, False, 1024, 128),
+                                                   (2, 12, 4, 16384, False, 512, 64)])
+def test_items_of_one_kv_head_and_q_block_are_adjacent(B, Hq, Hkv, N, causal, W, L):
+    # The pairs of one kv head at one q-block read the same K/V tiles in the same
+    # order; as consecutive items they go to neighbouring CTAs of the same round and
+    # run in lockstep, so each tile comes from DRAM once for all of them.
+    rec = tm.tm_debug_schedule(B, Hq, Hkv, N, causal, 64, W, L, 148)
+    G = Hq // Hkv
+    groups = {}
+    for c, item, qb, h0, nv, t0, t1 in rec:
+        groups.setdefault((qb, h0 // G), []).append(item)
+    npairs = (G + 1) // 2
+    for key, items in groups.items():
+        assert len(items) == npairs
+        assert max(items) - min(items) == npairs - 1, (key, sorted(items))
