@@ -893,7 +893,7 @@ __global__ void __launch_bounds__(128, 1)
   uint64_t* bar_mma = bar_load + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_load + 2);
   int* abort_flag = reinterpret_cast<int*>(bar_load + 3);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     mbar_init(bar_load, 1);
     mbar_init(bar_mma, 1);
