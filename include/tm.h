@@ -133,6 +133,26 @@ TM_API int tm_trianglemix_attn_fwd_ws(const void* q, const void* k, const void* 
                                       long long workspace_bytes, void* stream);
 
 /*
+ * tm_trianglemix_attn_fwd with the split schedule, for callers that cannot
+ * hand the library device memory: the paper has no counterpart. Instead of a
+ * caller workspace it uses a fixed scratch array of TM_NOALLOC_SCRATCH_BYTES
+ * (16 MiB) per device that the library's module holds; its address is looked
+ * up once per device (cudaGetSymbolAddress). The call allocates and frees
+ * nothing. A problem whose split schedule needs more scratch than that (as
+ * reported by tm_attn_workspace_size on this device) is rejected with
+ * TM_ERR_UNSUPPORTED before anything is enqueued; problems needing none run
+ * without touching the scratch. Each call clears the arrival counters it
+ * uses (an async memset on `stream`) before its kernel.
+ * Calls that overlap in time on one device race on the scratch and give
+ * undefined results: issue them on one stream, or order them otherwise.
+ */
+#define TM_NOALLOC_SCRATCH_BYTES (16LL << 20)
+TM_API int tm_trianglemix_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o,
+                                           int B, int Hq, int Hkv, int N, int D, float scale,
+                                           int S, int W, int L, int layer, int tri_start,
+                                           void* stream);
+
+/*
  * Number of kept (i, j) pairs of one (batch, head) of the triangle pattern:
  * sum over rows of min(i+1, W) + max(0, min(S, i+1-W)) for i < N-L and i+1
  * otherwise. Host only. Returns -1 on a bad argument.

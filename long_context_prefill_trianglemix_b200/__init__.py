@@ -27,7 +27,7 @@ EXPORTED = (
     "tm_triangle_kept_pairs", "tm_kept_tiles", "tm_triangle_tile_list", "tm_tile_list",
     "tm_debug_dump_tiles", "tm_debug_mma_probe", "tm_debug_schedule", "tm_get_device_status",
     "tm_status_string", "tm_attn_workspace_size", "tm_causal_attn_fwd_ws", "tm_triangle_attn_fwd_ws",
-    "tm_trianglemix_attn_fwd_ws",
+    "tm_trianglemix_attn_fwd_ws", "tm_trianglemix_attn_fwd_noalloc",
 )
 
 
@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
                                              vp, cll, vp]),
             "tm_trianglemix_attn_fwd_ws": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci,
                                                 ci, ci, ci, vp, cll, vp]),
+            "tm_trianglemix_attn_fwd_noalloc": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci,
+                                                     ci, ci, ci, ci, vp]),
             "tm_get_device_status": (ci, [vp]),
             "tm_status_string": (ctypes.c_char_p, [ci]),
         }
@@ -146,6 +148,16 @@ def tm_trianglemix_attn_fwd_ws(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L, lay
     return _check("tm_trianglemix_attn_fwd_ws", lib().tm_trianglemix_attn_fwd_ws(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, Hkv, N, D, scale, S, W, L, layer, tri_start,
         _ptr(workspace), int(workspace_bytes), _stream(stream)))
+
+
+def tm_trianglemix_attn_fwd_noalloc(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L, layer,
+                                    tri_start, stream=None):
+    return _check("tm_trianglemix_attn_fwd_noalloc", lib().tm_trianglemix_attn_fwd_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, Hkv, N, D, scale, S, W, L, layer, tri_start,
+        _stream(stream)))
+
+
+TM_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 def tm_attn_workspace_size(B, Hq, Hkv, N, D, causal, S, W, L, num_ctas=0) -> int:

@@ -5,6 +5,8 @@
 
 #include <cmath>
 #include <cstdint>
+#include <mutex>
+#include <vector>
 
 #include "tm.h"
 #include "tm_internal.h"
@@ -57,6 +59,29 @@ int validate_workspace(const void* q, const void* k, const void* v, const void* 
   if (overlaps(ws, ws_bytes, q, qbytes) || overlaps(ws, ws_bytes, o, qbytes) ||
       overlaps(ws, ws_bytes, k, kvbytes) || overlaps(ws, ws_bytes, v, kvbytes))
     return TM_ERR_INVALID_ARG;
+  return TM_OK;
+}
+
+// Scratch of tm_trianglemix_attn_fwd_noalloc: a fixed device array (one per
+// device, allocated with the module, never by a call) used as the split
+// workspace. Its address is looked up once per device.
+constexpr long long kScratchBytes = TM_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_split_scratch[kScratchBytes];
+
+std::mutex g_scratch_mutex;
+std::vector<void*> g_scratch_addr;  // per device; nullptr until looked up
+
+int scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return TM_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (static_cast<int>(g_scratch_addr.size()) <= dev) g_scratch_addr.resize(dev + 1, nullptr);
+  if (!g_scratch_addr[dev]) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_split_scratch) != cudaSuccess || !a) return TM_ERR_CUDA;
+    g_scratch_addr[dev] = a;
+  }
+  *out = g_scratch_addr[dev];
   return TM_OK;
 }
 
@@ -138,6 +163,27 @@ TM_API int tm_attn_workspace_size(int B, int Hq, int Hkv, int N, int D, int caus
     return TM_ERR_INVALID_ARG;
   return trimix::workspace_bytes(B, Hq, Hkv, N, D, trimix::make_pattern(N, causal, S, W, L),
                                  num_ctas, bytes);
+}
+
+TM_API int tm_trianglemix_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o,
+                                           int B, int Hq, int Hkv, int N, int D, float scale,
+                                           int S, int W, int L, int layer, int tri_start,
+                                           void* stream) {
+  if (layer < 0 || tri_start < 0) return TM_ERR_INVALID_ARG;
+  const int causal = layer < tri_start ? 1 : 0;
+  if (int rc = validate_common(q, k, v, o, B, Hq, Hkv, N, D, scale)) return rc;
+  if (!causal)
+    if (int rc = validate_pattern(S, W, L)) return rc;
+  const trimix::Pattern pat = causal ? trimix::make_pattern(N, 1, 0, 1, 0)
+                                     : trimix::make_pattern(N, 0, S, W, L);
+  long long need = 0;
+  if (int rc = trimix::workspace_bytes(B, Hq, Hkv, N, D, pat, 0, &need)) return rc;
+  if (need > kScratchBytes) return TM_ERR_UNSUPPORTED;  // larger than the fixed scratch
+  void* scratch = nullptr;
+  if (need > 0)
+    if (int rc = scratch_address(&scratch)) return rc;
+  return run(q, k, v, o, B, Hq, Hkv, N, D, scale, pat, scratch, need > 0 ? kScratchBytes : 0,
+             stream);
 }
 
 TM_API long long tm_triangle_kept_pairs(int N, int S, int W, int L) {
