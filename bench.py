@@ -293,7 +293,29 @@ def run_ours(args):
     torch.cuda.synchronize()
     e2e_ms = sum(ee[s][0].elapsed_time(ee[s][1]) for s in range(e2e_steps)) / e2e_steps
 
-    total_ms, tri_sum, e2e_ms = reduce_over_ranks([total_ms, tri_sum, e2e_ms], device="cuda")
+    # block-sparse shallow layer (next to the triangle path: a seeded vertical /
+    # slash / local block index, 128x128 blocks), timed on its own after the steps
+    bs_off, bs_idx = I.make_block_index(wl.B, wl.Hkv, wl.N, 0)
+    d_off = torch.from_numpy(bs_off).cuda()
+    d_idx = torch.from_numpy(bs_idx).cuda()
+
+    def sparse_call():
+        tm.tm_block_sparse_attn_fwd(dq, dk, dv, do, wl.B, wl.Hq, wl.Hkv, wl.N, wl.D, wl.scale,
+                                    d_off, d_idx, len(bs_idx), stream)
+
+    for _ in range(args.warmup):
+        sparse_call()
+    bs_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for s in range(args.steps):
+        bs_ev[s][0].record(stream)
+        sparse_call()
+        bs_ev[s][1].record(stream)
+    torch.cuda.synchronize()
+    bs_ms = sum(bs_ev[s][0].elapsed_time(bs_ev[s][1]) for s in range(args.steps))
+    bs_f = float(len(bs_idx)) * (wl.Hq // wl.Hkv) * 4.0 * BM * BN * wl.D
+
+    total_ms, tri_sum, e2e_ms, bs_ms = reduce_over_ranks([total_ms, tri_sum, e2e_ms, bs_ms],
+                                                         device="cuda")
 
     peaks = load_peaks()
     tri_avg = tri_sum / args.steps
@@ -327,6 +349,16 @@ def run_ours(args):
                 "h2d_bytes_per_step": int((dq.numel() + dk.numel() + dv.numel()) * 2),
                 "d2h_bytes_per_step": int(do.numel() * 2),
                 "what": "pinned host q,k,v -> device, triangle layer, output -> pinned host"},
+        "block_sparse": {
+            "what": "tm_block_sparse_attn_fwd, seeded block index (local 8, sink 1, vertical 32, "
+                    "slash 8 blocks per list), timed separately after the steps",
+            "ms": bs_ms / args.steps,
+            "tflops_kept_tiles": bs_f / (bs_ms / args.steps * 1e-3) / 1e12,
+            "kept_tiles": int(len(bs_idx)) * (wl.Hq // wl.Hkv),
+            "density_vs_causal": len(bs_idx) / (wl.B * wl.Hkv * ((wl.N + BM - 1) // BM)
+                                                * ((wl.N + BM - 1) // BM + 1) / 2),
+            "speedup_vs_causal": (sum(cau_ms) / args.steps) / (bs_ms / args.steps),
+        },
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
         "device_status": tm.status_string(status),

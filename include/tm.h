@@ -94,6 +94,39 @@ TM_API int tm_trianglemix_attn_fwd(const void* q, const void* k, const void* v, 
                                    int L, int layer, int tri_start, void* stream);
 
 /*
+ * Block-sparse causal attention from a caller's block index, on the same
+ * kernels: the visited tiles of each q-block come from the index instead of a
+ * closed form, the way the FlashPrefill summary (section 2.3) jumps straight
+ * to the selected blocks instead of testing every block. Meant for the
+ * shallow layers that the TriangleMix blog post (section 介绍, last paragraph)
+ * leaves to dynamic sparse methods; pattern discovery produces such an index.
+ *   keep(i, j) = j <= i  and  j < N  and  j / TM_BLOCK_N is listed for
+ *                (batch, kv head of the row's q head, q-block i / TM_BLOCK_M).
+ * Index (DEVICE memory, int32, CSR): with nqb = ceil(N / TM_BLOCK_M) and
+ * r = (b * Hkv + g) * nqb + qb, block_offsets[r] .. block_offsets[r + 1]
+ * (B * Hkv * nqb + 1 entries, non-decreasing, within [0, nnz]) delimit the
+ * k-blocks of that q-block in block_indices[0 .. nnz), which should be strictly
+ * ascending in [0, qb]. All q heads of a kv head's group share its lists.
+ * Offsets are clamped to [0, nnz] and entries outside [0, qb] are visited as
+ * fully masked tiles, so a malformed index yields wrong values, never an
+ * access outside q, k, v, o or the index; a duplicated entry counts its keys
+ * twice. A row that keeps no key is written as zeros. The index is read by the
+ * kernel (no host synchronisation).
+ * tm_trianglemix_sparse_attn_fwd is the layer schedule with this as the
+ * shallow layers: layer < tri_start runs the block-sparse call with the
+ * index, layer >= tri_start runs tm_triangle_attn_fwd (the index is ignored).
+ */
+TM_API int tm_block_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o, int B,
+                                    int Hq, int Hkv, int N, int D, float scale,
+                                    const int* block_offsets, const int* block_indices,
+                                    long long nnz, void* stream);
+TM_API int tm_trianglemix_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o,
+                                          int B, int Hq, int Hkv, int N, int D, float scale,
+                                          int S, int W, int L, int layer, int tri_start,
+                                          const int* block_offsets, const int* block_indices,
+                                          long long nnz, void* stream);
+
+/*
  * Split schedule for the long q-blocks. The last L query rows of the triangle
  * (and the last rows of causal attention) see every earlier key, so one of
  * their items can cost more than a CTA's share of the launch when B * Hq is

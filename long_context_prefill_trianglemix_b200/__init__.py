@@ -27,7 +27,8 @@ EXPORTED = (
     "tm_triangle_kept_pairs", "tm_kept_tiles", "tm_triangle_tile_list", "tm_tile_list",
     "tm_debug_dump_tiles", "tm_debug_mma_probe", "tm_debug_schedule", "tm_get_device_status",
     "tm_status_string", "tm_attn_workspace_size", "tm_causal_attn_fwd_ws", "tm_triangle_attn_fwd_ws",
-    "tm_trianglemix_attn_fwd_ws", "tm_trianglemix_attn_fwd_noalloc",
+    "tm_trianglemix_attn_fwd_ws", "tm_trianglemix_attn_fwd_noalloc", "tm_block_sparse_attn_fwd",
+    "tm_trianglemix_sparse_attn_fwd",
 )
 
 
@@ -73,6 +74,10 @@ def lib() -> ctypes.CDLL:
                                                 ci, ci, ci, vp, cll, vp]),
             "tm_trianglemix_attn_fwd_noalloc": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci,
                                                      ci, ci, ci, ci, vp]),
+            "tm_block_sparse_attn_fwd": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp, vp, cll,
+                                              vp]),
+            "tm_trianglemix_sparse_attn_fwd": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci,
+                                                    ci, ci, ci, vp, vp, cll, vp]),
             "tm_get_device_status": (ci, [vp]),
             "tm_status_string": (ctypes.c_char_p, [ci]),
         }
@@ -158,6 +163,20 @@ def tm_trianglemix_attn_fwd_noalloc(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L
 
 
 TM_NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def tm_block_sparse_attn_fwd(q, k, v, o, B, Hq, Hkv, N, D, scale, block_offsets, block_indices,
+                             nnz, stream=None):
+    return _check("tm_block_sparse_attn_fwd", lib().tm_block_sparse_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, Hkv, N, D, scale, _ptr(block_offsets),
+        _ptr(block_indices), int(nnz), _stream(stream)))
+
+
+def tm_trianglemix_sparse_attn_fwd(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L, layer,
+                                   tri_start, block_offsets, block_indices, nnz, stream=None):
+    return _check("tm_trianglemix_sparse_attn_fwd", lib().tm_trianglemix_sparse_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, Hkv, N, D, scale, S, W, L, layer, tri_start,
+        _ptr(block_offsets), _ptr(block_indices), int(nnz), _stream(stream)))
 
 
 def tm_attn_workspace_size(B, Hq, Hkv, N, D, causal, S, W, L, num_ctas=0) -> int:

@@ -86,8 +86,12 @@ int scratch_address(void** out) {
 }
 
 int run(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv, int N, int D,
-        float scale, const trimix::Pattern& pat, void* ws, long long ws_bytes, void* stream) {
+        float scale, const trimix::Pattern& pat, void* ws, long long ws_bytes, void* stream,
+        const int* bs_off = nullptr, const int* bs_idx = nullptr, long long bs_nnz = 0) {
   trimix::LaunchArgs a;
+  a.bs_off = bs_off;
+  a.bs_idx = bs_idx;
+  a.bs_nnz = bs_nnz;
   a.q = q; a.k = k; a.v = v; a.o = o;
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.N = N; a.D = D;
   a.scale = scale;
@@ -151,6 +155,32 @@ TM_API int tm_trianglemix_attn_fwd(const void* q, const void* k, const void* v, 
                                    int layer, int tri_start, void* stream) {
   return tm_trianglemix_attn_fwd_ws(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L, layer,
                                     tri_start, nullptr, 0, stream);
+}
+
+TM_API int tm_block_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o, int B,
+                                    int Hq, int Hkv, int N, int D, float scale,
+                                    const int* block_offsets, const int* block_indices,
+                                    long long nnz, void* stream) {
+  if (int rc = validate_common(q, k, v, o, B, Hq, Hkv, N, D, scale)) return rc;
+  if (!block_offsets || nnz < 0 || nnz > (1LL << 31) - 1 || (nnz > 0 && !block_indices))
+    return TM_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(block_offsets) & 3u) ||
+      (reinterpret_cast<uintptr_t>(block_indices) & 3u))
+    return TM_ERR_INVALID_ARG;
+  return run(q, k, v, o, B, Hq, Hkv, N, D, scale, trimix::make_pattern(N, 1, 0, 1, 0), nullptr, 0,
+             stream, block_offsets, nnz > 0 ? block_indices : block_offsets, nnz);
+}
+
+TM_API int tm_trianglemix_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o,
+                                          int B, int Hq, int Hkv, int N, int D, float scale,
+                                          int S, int W, int L, int layer, int tri_start,
+                                          const int* block_offsets, const int* block_indices,
+                                          long long nnz, void* stream) {
+  if (layer < 0 || tri_start < 0) return TM_ERR_INVALID_ARG;
+  if (layer < tri_start)
+    return tm_block_sparse_attn_fwd(q, k, v, o, B, Hq, Hkv, N, D, scale, block_offsets,
+                                    block_indices, nnz, stream);
+  return tm_triangle_attn_fwd(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L, stream);
 }
 
 TM_API int tm_attn_workspace_size(int B, int Hq, int Hkv, int N, int D, int causal, int S, int W,

@@ -162,6 +162,12 @@ struct AttnParams {
   int nsplit;
   float* ws_rec;
   int* ws_cnt;
+  // Block-sparse launches (bs_off != nullptr): the tile list of item (b, kv
+  // head g, q-block qb) is bs_idx[bs_off[r] .. bs_off[r + 1]), r = (b * Hkv +
+  // g) * nqb + qb, offsets clamped to [0, bs_nnz]; pat is the causal pattern.
+  const int* bs_off;
+  const int* bs_idx;
+  int bs_nnz;
 };
 
 __host__ __device__ __forceinline__ int big_count(const AttnParams& p, int c, int g) {
@@ -246,6 +252,40 @@ __host__ __device__ __forceinline__ Item decode_piece(const AttnParams& p, int b
     it.hunit = qi * p.units + u;
   }
   return it;
+}
+
+// The tile list of one item: the closed form of the pattern, or a run of the
+// caller's block index. Index entries are clamped to [-1, nqb]: TMA reads
+// zeros outside the tensor, and the softmax masks such tiles completely, so a
+// malformed index gives masked tiles, never an access outside q, k or v.
+struct TileSrc {
+  BlockTiles bt;
+  const int* idx;  // nullptr: closed form
+  int n, nkb;
+  __device__ __forceinline__ int count() const { return idx ? n : bt.count(); }
+  __device__ __forceinline__ int kb(int t) const {
+    if (!idx) return bt.kb(t);
+    const int v = __ldg(idx + t);
+    return v < -1 ? -1 : (v > nkb ? nkb : v);
+  }
+};
+
+__device__ __forceinline__ TileSrc tile_src(const AttnParams& p, const Item& it) {
+  TileSrc s;
+  s.idx = nullptr;
+  s.n = 0;
+  s.nkb = p.nqb;
+  if (p.bs_off) {
+    const long long r = (static_cast<long long>(it.b) * p.Hkv + it.g) * p.nqb + it.qb;
+    const int o0 = imin(imax(__ldg(p.bs_off + r), 0), p.bs_nnz);
+    const int o1 = imin(imax(__ldg(p.bs_off + r + 1), o0), p.bs_nnz);
+    s.idx = p.bs_idx + o0;
+    s.n = o1 - o0;
+    s.bt.n_a = s.bt.b_lo = s.bt.n_b = 0;
+  } else {
+    s.bt = block_tiles(p.pat, it.qb, BM, BN);
+  }
+  return s;
 }
 
 // Walks one CTA's work (the same sequence as work_item) without an integer
@@ -429,7 +469,9 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, Bars<Cfg<D>::
   cur.init(p, blockIdx.x, gridDim.x);
   while (ok && !cur.done()) {
     const Item it = cur.next(p);
-    const BlockTiles bt = block_tiles(p.pat, it.qb, BM, BN);
+    const TileSrc bt = tile_src(p, it);
+    const int t_end = imin(bt.count(), it.t1);
+    if (t_end <= it.t0) continue;  // an empty block-sparse list: nothing to load
     if (!(ok = wait_bar(&bars->q_empty, (it_cnt & 1u) ^ 1u, abort_flag, kSiteQEmpty))) break;
     mbar_arrive_expect_tx(&bars->q_full, (1 + it.v1) * Cfg<D>::kTileBytes);
 #pragma unroll
@@ -440,7 +482,6 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, Bars<Cfg<D>::
                     it.h0 + 1, it.qb * BM, it.b);
     }
     ++it_cnt;
-    const int t_end = imin(bt.count(), it.t1);
     for (int t = it.t0; ok && t < t_end; ++t) {
       const int kb = bt.kb(t);
 #pragma unroll
@@ -492,7 +533,8 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStag
   cur.init(p, blockIdx.x, gridDim.x);
   while (ok && !cur.done()) {
     const Item it = cur.next(p);
-    const int T = imin(block_tiles(p.pat, it.qb, BM, BN).count(), it.t1) - it.t0;
+    const int T = imin(tile_src(p, it).count(), it.t1) - it.t0;
+    if (T <= 0) continue;  // an empty block-sparse list
     const bool v1 = it.v1 != 0;
     TM_WAIT(&bars->q_full, it_cnt & 1u, kSiteQFull);
     ++it_cnt;
@@ -647,7 +689,7 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
   while (!cur.done()) {
     const Item it = cur.next(p);
     if (wg == 1 && !it.v1) continue;
-    const BlockTiles bt = block_tiles(pat, it.qb, BM, BN);
+    const TileSrc bt = tile_src(p, it);
     const int T = imin(bt.count(), it.t1) - it.t0;
     const int i = it.qb * BM + r;  // query row of this thread
     // kept keys of row i: [0, sink_hi) U [band_lo, hi)
@@ -657,8 +699,9 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
     const int band_lo = full_row ? hi : imax(0, i - pat.W + 1);
     float m_run = -INFINITY, l_run = 0.f;
     for (int t = 0; t < T; ++t) {
-      const int kb = bt.kb(it.t0 + t);
-      const bool need_mask = tile_needs_mask(pat, it.qb, kb, BM, BN) != 0;
+      const int kb = bt.kb(it.t0 + t);  // read before the wait, which hides its latency
+      const bool bad = kb < 0;          // a clamped negative index entry: fully masked
+      const bool need_mask = bad || tile_needs_mask(pat, it.qb, kb, BM, BN) != 0;
       bool ok = wait_bar(&bars->s_full[wg], s_cnt & 1u, abort_flag, kSiteSFull);
       ++s_cnt;
       if (!__all_sync(0xffffffffu, ok)) return;
@@ -672,7 +715,7 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
       reg_fence(sr[3]);
       if (need_mask) {
         // keep bits of this row for the tile's 128 columns, then -inf elsewhere
-        const int c0 = kb * BN;
+        const int c0 = bad ? (1 << 30) : kb * BN;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const uint32_t keep = range_bits(sink_hi - c0 - 32 * c) |
@@ -751,18 +794,25 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
     }
     // epilogue: O / l -> bf16 -> this warp's 128B-swizzled staging slot (32 rows x
     // 64 columns at a time) -> one TMA store per half; rows past N are clipped.
-    bool ok = wait_bar(&bars->o_full[wg], o_cnt & 1u, abort_flag, kSiteOFull);
-    ++o_cnt;
-    if (!__all_sync(0xffffffffu, ok)) return;
-    tc_fence_after();
     uint32_t orr[D / 32][32];
+    if (T > 0) {
+      bool ok = wait_bar(&bars->o_full[wg], o_cnt & 1u, abort_flag, kSiteOFull);
+      ++o_cnt;
+      if (!__all_sync(0xffffffffu, ok)) return;
+      tc_fence_after();
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + 32 * c, orr[c]);
-    tmem_wait_ld(orr[0]);
+      for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + 32 * c, orr[c]);
+      tmem_wait_ld(orr[0]);
 #pragma unroll
-    for (int c = 1; c < D / 32; ++c) reg_fence(orr[c]);
-    tc_fence_before();
-    mbar_arrive(&bars->o_empty[wg]);
+      for (int c = 1; c < D / 32; ++c) reg_fence(orr[c]);
+      tc_fence_before();
+      mbar_arrive(&bars->o_empty[wg]);
+    } else {  // an empty block-sparse list: the rows keep no key and come out as zeros
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c)
+#pragma unroll
+        for (int x = 0; x < 32; ++x) orr[c][x] = 0u;
+    }
     if (it.split >= 0 && !merge_split<D>(p, it, wg, wq, lane, orr, m_run, l_run)) continue;
     const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
     const uint32_t slot = smem_addr(smem + Cfg<D>::kStageOff) + (wg * 4 + wq) * Cfg<D>::kStageSlotBytes;
@@ -1045,7 +1095,7 @@ int encode_bnhd(CUtensorMap* m, const void* base, int B, int N, int H, int D, in
 // Fills the geometry and the persistent work split of *p; returns the grid
 // size. split: heavy items may be cut into pieces (the caller has workspace).
 int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ctas, bool split,
-                   AttnParams* p) {
+                   AttnParams* p, bool sparse = false) {
   p->B = B; p->Hq = Hq; p->Hkv = Hkv; p->N = N;
   p->G = Hq / Hkv;
   p->npairs = (p->G + 1) / 2;
@@ -1055,6 +1105,9 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
   p->ws_rec = nullptr;
   p->ws_cnt = nullptr;
   p->pair_rot = 0;
+  p->bs_off = nullptr;
+  p->bs_idx = nullptr;
+  p->bs_nnz = 0;
   // Persistent grid. Item cost = (visited tiles + fixed per-item overhead,
   // about the pipeline fill/drain and epilogue) x Q tiles of the item; it is
   // used to find the heavy q-blocks, how finely to cut them, and how many
@@ -1071,8 +1124,10 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
   // heavy q-blocks: from the top, while an item of the block costs more than a
   // quarter of a CTA's share (at most 8 big items per CTA)
   const long long item_q = p->G >= 2 ? 2 : 1;
+  // (block-sparse launches: costs are in device memory, every item is dealt
+  // in the strided rounds, q-blocks from the last)
   int n_hqb = 0;
-  while (n_hqb < p->nqb - 1 && 4.0 * qcost[p->nqb - 1 - n_hqb] * item_q > target &&
+  while (!sparse && n_hqb < p->nqb - 1 && 4.0 * qcost[p->nqb - 1 - n_hqb] * item_q > target &&
          static_cast<long long>(n_hqb + 1) * p->units <= 8LL * grid)
     ++n_hqb;
   p->n_hqb = n_hqb;
@@ -1081,7 +1136,7 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
   // share into ns pieces (ns from the heaviest, so its pieces fit that share),
   // each of at least kMinPieceTiles tiles, at most 8 big pieces per CTA.
   int ns = 1, n_sqb = 0;
-  if (split && n_hqb > 0) {
+  if (split && !sparse && n_hqb > 0) {
     const double heavy = static_cast<double>(qcost[p->nqb - 1] * item_q);
     ns = static_cast<int>(std::ceil(heavy / (kSplitShare * target)));
     ns = std::min(ns, std::max(1, block_tiles(p->pat, p->nqb - 1, BM, BN).count() / kMinPieceTiles));
@@ -1172,8 +1227,15 @@ int launch_attention_d(const LaunchArgs& a, DeviceInfo* di) {
     return TM_ERR_CUDA;
 
   AttnParams p;
-  const int grid = build_schedule(a.B, a.Hq, a.Hkv, a.N, a.pat, di->sms, a.ws != nullptr, &p);
+  const bool sparse = a.bs_off != nullptr;
+  const int grid =
+      build_schedule(a.B, a.Hq, a.Hkv, a.N, a.pat, di->sms, a.ws != nullptr, &p, sparse);
   p.sl2 = a.scale * 1.4426950408889634f;
+  if (sparse) {
+    p.bs_off = a.bs_off;
+    p.bs_idx = a.bs_idx;
+    p.bs_nnz = static_cast<int>(a.bs_nnz);
+  }
   const WsLayout w = ws_layout(p, D);
   if (w.total > 0) {
     if (a.ws_bytes < w.total) return TM_ERR_INVALID_ARG;

@@ -21,6 +21,9 @@ struct LaunchArgs {
   Pattern pat;
   void* ws;           // split workspace (device), or nullptr: no item is split
   long long ws_bytes;
+  const int* bs_off;  // block-sparse index (device CSR), or nullptr: pat's tile list
+  const int* bs_idx;
+  long long bs_nnz;
   void* stream;
 };
 

@@ -223,3 +223,59 @@ def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
     r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
     r[nan] = ((u[nan] >> 16) | 0x40).astype(np.uint16)
     return r
+
+
+@dataclass(frozen=True)
+class BlockIndexRecipe:
+    """Structure of a synthetic block index (128 x 128 blocks) for the
+    block-sparse shallow layers. The FlashPrefill summary (section 2.1) names
+    the structures such indices hold: vertical (key blocks every query block
+    attends to), slash (fixed distances below the diagonal) and scattered
+    blocks; the first block (sinks) and the blocks next to the diagonal are
+    kept by every such method. Counts are per (batch, kv head) for vertical
+    and slash, per q-block for the local band; ``p_block`` is the chance that
+    any other causal block is kept."""
+    local: int = 8        # blocks qb-local+1 .. qb
+    sink: int = 1         # blocks 0 .. sink-1
+    vertical: int = 32    # seeded key blocks kept by every later q-block
+    slash: int = 8        # seeded distances d: block qb - d
+    p_block: float = 0.0  # independent chance of any remaining block
+
+
+def make_block_index(B: int, Hkv: int, N: int, seed: int, recipe: BlockIndexRecipe = None,
+                     BM: int = 128):
+    """CSR block index: offsets int32 [B * Hkv * nqb + 1], indices int32 [nnz],
+    each list strictly ascending within [0, qb]. Draws only index structure."""
+    recipe = recipe or BlockIndexRecipe()
+    nqb = (N + BM - 1) // BM
+    lists = []
+    for b in range(B):
+        for g in range(Hkv):
+            stream = 3000 + 64 * (b * Hkv + g)
+            vert = {int(_uniform(seed, stream, n) * nqb) for n in range(recipe.vertical)}
+            dist = {1 + int(_uniform(seed, stream + 1, n) * max(1, nqb - 1))
+                    for n in range(recipe.slash)}
+            rnd_key = _mix64(_mix64(seed) ^ _mix64(stream + 2))
+            for qb in range(nqb):
+                kb = set(range(max(0, qb - recipe.local + 1), qb + 1))
+                kb |= set(range(min(recipe.sink, qb + 1)))
+                kb |= {c for c in vert if c <= qb}
+                kb |= {qb - d for d in dist if d <= qb}
+                if recipe.p_block > 0:
+                    rng = np.random.default_rng((rnd_key + qb) & _M64)
+                    extra = np.flatnonzero(rng.random(qb + 1) < recipe.p_block)
+                    kb |= set(extra.tolist())
+                lists.append(sorted(kb))
+    offsets = np.zeros(len(lists) + 1, np.int32)
+    offsets[1:] = np.cumsum([len(x) for x in lists])
+    indices = np.fromiter((c for x in lists for c in x), dtype=np.int32, count=int(offsets[-1]))
+    return offsets, indices
+
+
+def full_causal_index(B: int, Hkv: int, N: int, BM: int = 128):
+    """CSR index listing every causal block (block-sparse = causal attention)."""
+    nqb = (N + BM - 1) // BM
+    per = [list(range(qb + 1)) for qb in range(nqb)] * (B * Hkv)
+    offsets = np.zeros(len(per) + 1, np.int32)
+    offsets[1:] = np.cumsum([len(x) for x in per])
+    return offsets, np.fromiter((c for x in per for c in x), np.int32, count=int(offsets[-1]))

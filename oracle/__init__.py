@@ -44,6 +44,10 @@ def _load():
         lib.oracle_attention.restype = c_int
         lib.oracle_attention.argtypes = [vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_dbl,
                                          c_int, c_int, c_int, c_int, vp, c_ll, vp, vp, c_int]
+        lib.oracle_block_sparse_attention.restype = c_int
+        lib.oracle_block_sparse_attention.argtypes = [
+            vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_dbl, c_int, c_int, vp, vp, c_ll, vp,
+            c_ll, vp, c_int]
         for name in ("oracle_tile_list_bruteforce", "oracle_tile_list_rows"):
             f = getattr(lib, name)
             f.restype = c_int
@@ -125,3 +129,31 @@ def attention(q, k, v, B, Hq, Hkv, N, D, scale, causal, S=0, W=1, L=0, rows=None
     if rc != 0:
         raise ValueError("oracle_attention: bad argument")
     return (out, rs) if with_rowsum else out
+
+
+def block_sparse_attention(q, k, v, B, Hq, Hkv, N, D, scale, offsets, indices, rows=None, BM=128,
+                           BS=128, nthreads=None):
+    """fp64 block-sparse causal attention from a CSR block index.
+
+    offsets: int32 [B * Hkv * ceil(N / BM) + 1]; indices: int32 [nnz] (k-block
+    numbers of each (batch, kv head, q-block)). Returns out [B, nrows, Hq, D].
+    """
+    lib = _load()
+    for a in (q, k, v):
+        assert a.dtype == np.uint16 and a.flags.c_contiguous
+    off = np.ascontiguousarray(offsets, dtype=np.int32)
+    idx = np.ascontiguousarray(indices, dtype=np.int32)
+    assert off.size == B * Hkv * ((N + BM - 1) // BM) + 1
+    if rows is None:
+        nrows, rows_ptr = N, None
+    else:
+        rows_arr = np.ascontiguousarray(rows, dtype=np.int64)
+        nrows, rows_ptr = len(rows_arr), rows_arr.ctypes.data
+    out = np.zeros((B, nrows, Hq, D), np.float64)
+    rc = lib.oracle_block_sparse_attention(
+        q.ctypes.data, k.ctypes.data, v.ctypes.data, B, Hq, Hkv, N, D, float(scale), BM, BS,
+        off.ctypes.data, idx.ctypes.data if idx.size else None, int(idx.size), rows_ptr, nrows,
+        out.ctypes.data, nthreads or hardware_threads())
+    if rc != 0:
+        raise ValueError("oracle_block_sparse_attention: bad argument")
+    return out

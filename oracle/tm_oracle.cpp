@@ -29,7 +29,10 @@
 //   * L = N or S + W >= N gives causal attention;
 //   * the last L rows equal the causal rows; rows sum to 1;
 //   * S=0, W=1, L=0 gives o_i = v_i; q = 0 gives the mean of v over K_i;
-//   * causal and masked rows match a library softmax-attention routine.
+//   * causal and masked rows match a library softmax-attention routine;
+//   * block-sparse: every causal block listed gives causal attention exactly;
+//     q = 0 gives the mean of v over the kept keys; rows match the library
+//     routine under a block mask built independently; empty lists give 0.
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
@@ -203,6 +206,88 @@ int oracle_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, in
           double sum = 0.0;
           for (size_t t = 0; t < idx.size(); ++t) sum += s[t] / l;
           rowsum[(b * nrows + r) * Hq + hq] = sum;
+        }
+      }
+    }
+  });
+  return 0;
+}
+
+// Block-sparse causal attention in fp64 (the shallow-layer counterpart the
+// TriangleMix blog post, section 介绍, leaves to dynamic sparse methods; the
+// block index is the input format of the FlashPrefill summary, section 2.3):
+//
+//   keep(i, j) = j <= i  and  j / BS is listed for (b, g, i / BM)
+//
+// with the list of (b, kv head g, q-block qb) = the entries
+// indices[offsets[r] .. offsets[r+1]), r = (b * Hkv + g) * nqb + qb,
+// nqb = ceil(N / BM), read as a set of k-block numbers (entries that name no
+// block of keys j <= i keep nothing). Each mask row is built explicitly from
+// that definition; the attention is the same fp64 computation as above, and a
+// row that keeps no key is 0. Returns 0, or -1 on a bad argument (offsets
+// decreasing or outside [0, nnz]).
+int oracle_block_sparse_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B,
+                                  int Hq, int Hkv, int N, int D, double scale, int BM, int BS,
+                                  const int* offsets, const int* indices, long long nnz,
+                                  const long long* rows, long long nrows, double* out,
+                                  int nthreads) {
+  if (!q || !k || !v || !out || !offsets || B < 1 || Hq < 1 || Hkv < 1 || N < 1 || D < 1 ||
+      Hq % Hkv != 0 || BM < 1 || BS < 1 || nnz < 0 || (nnz > 0 && !indices))
+    return -1;
+  const long long nqb = (N + BM - 1) / BM, nrec = (long long)B * Hkv * nqb;
+  for (long long r = 0; r <= nrec; ++r)
+    if (offsets[r] < 0 || offsets[r] > nnz || (r > 0 && offsets[r] < offsets[r - 1])) return -1;
+  if (!rows) nrows = N;
+  if (nrows < 0) return -1;
+  for (long long r = 0; rows && r < nrows; ++r)
+    if (rows[r] < 0 || rows[r] >= N) return -1;
+  const int G = Hq / Hkv;
+  const long long units = (long long)B * nrows;
+  parallel_for(units, nthreads, [&](long long ub, long long ue) {
+    std::vector<unsigned char> listed, m(static_cast<size_t>(N));
+    std::vector<long long> idx;
+    std::vector<double> s, qrow(static_cast<size_t>(D)), o(static_cast<size_t>(D));
+    for (long long u = ub; u < ue; ++u) {
+      const long long b = u / nrows, r = u % nrows;
+      const long long i = rows ? rows[r] : r;
+      for (int g = 0; g < Hkv; ++g) {
+        // explicit mask row of (b, g, i)
+        const long long rec = (b * Hkv + g) * nqb + i / BM;
+        listed.assign(static_cast<size_t>((N + BS - 1) / BS), 0);
+        for (long long e = offsets[rec]; e < offsets[rec + 1]; ++e)
+          if (indices[e] >= 0 && indices[e] < (long long)listed.size()) listed[size_t(indices[e])] = 1;
+        for (long long j = 0; j < N; ++j) m[size_t(j)] = (j <= i && listed[size_t(j / BS)]) ? 1 : 0;
+        idx.clear();
+        for (long long j = 0; j < N; ++j)
+          if (m[size_t(j)]) idx.push_back(j);
+        s.resize(idx.size());
+        for (int hq = g * G; hq < (g + 1) * G; ++hq) {
+          double* op = out + ((b * nrows + r) * Hq + hq) * (long long)D;
+          if (idx.empty()) {
+            for (int d = 0; d < D; ++d) op[d] = 0.0;
+            continue;
+          }
+          const uint16_t* qp = q + ((b * N + i) * Hq + hq) * (long long)D;
+          for (int d = 0; d < D; ++d) qrow[size_t(d)] = bf16_to_double(qp[d]);
+          double mx = -std::numeric_limits<double>::infinity();
+          for (size_t t = 0; t < idx.size(); ++t) {
+            const uint16_t* kp = k + ((b * N + idx[t]) * Hkv + g) * (long long)D;
+            double acc = 0.0;
+            for (int d = 0; d < D; ++d) acc += qrow[size_t(d)] * bf16_to_double(kp[d]);
+            s[t] = scale * acc;
+            mx = std::max(mx, s[t]);
+          }
+          double l = 0.0;
+          for (size_t t = 0; t < idx.size(); ++t) {
+            s[t] = std::exp(s[t] - mx);
+            l += s[t];
+          }
+          std::fill(o.begin(), o.end(), 0.0);
+          for (size_t t = 0; t < idx.size(); ++t) {
+            const uint16_t* vp = v + ((b * N + idx[t]) * Hkv + g) * (long long)D;
+            for (int d = 0; d < D; ++d) o[size_t(d)] += s[t] * bf16_to_double(vp[d]);
+          }
+          for (int d = 0; d < D; ++d) op[d] = o[size_t(d)] / l;
         }
       }
     }

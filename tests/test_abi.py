@@ -162,3 +162,19 @@ def test_workspace_size_arguments():
         tm.TM_ERR_INVALID_ARG
     assert L.tm_attn_workspace_size(1, 4, 1, 4096, 128, 0, 16, 64, 64, 148, ctypes.byref(n)) == 0
     assert n.value >= 0
+
+
+def test_block_sparse_validation():
+    L = tm.lib()
+    args = (FAKE, FAKE, FAKE, FAKE + 0x100000, 1, 4, 4, 64, 64, 0.1)
+    off = FAKE + 0x200000
+    assert L.tm_block_sparse_attn_fwd(*args, None, off, 4, None) == tm.TM_ERR_INVALID_ARG
+    assert L.tm_block_sparse_attn_fwd(*args, off, None, 4, None) == tm.TM_ERR_INVALID_ARG
+    assert L.tm_block_sparse_attn_fwd(*args, off, off, -1, None) == tm.TM_ERR_INVALID_ARG
+    assert L.tm_block_sparse_attn_fwd(*args, off + 2, off, 4, None) == tm.TM_ERR_INVALID_ARG
+    assert L.tm_block_sparse_attn_fwd(*args, off, off, 1 << 31, None) == tm.TM_ERR_INVALID_ARG
+    assert L.tm_trianglemix_sparse_attn_fwd(*args, 4, 8, 2, -1, 1, off, off, 4,
+                                            None) == tm.TM_ERR_INVALID_ARG
+    # the triangle branch ignores the index but still checks the pattern
+    assert L.tm_trianglemix_sparse_attn_fwd(*args, 4, 0, 2, 3, 1, None, None, 0,
+                                            None) == tm.TM_ERR_INVALID_ARG
