@@ -127,6 +127,42 @@ TM_API int tm_trianglemix_sparse_attn_fwd(const void* q, const void* k, const vo
                                           long long nnz, void* stream);
 
 /*
+ * Block pattern discovery: builds the block index of tm_block_sparse_attn_fwd
+ * on the GPU, after the FlashPrefill summary (section 2.1: uniformly spread
+ * probe queries against average-pooled key blocks; section 2.2: keep the
+ * blocks whose score reaches alpha times the best score of their query block,
+ * no top-k / top-p sort). For batch b, kv head g and q-block I (rows
+ * [r0, r1)):
+ *   kbar_J       = mean of k[b, j, g, :] over the keys of block J
+ *   probe rows   max(r0, r0 + ((p + 1) (r1 - r0)) / probes - 1), p = 0 .. probes-1,
+ *                in each q head h of g's group
+ *   pi_{h,p}(J)  = softmax over J in [0, I] of scale * q[b, row_p, h, :] . kbar_J
+ *   Score(I, J)  = mean over (h, p) of pi_{h,p}(J)
+ *   list(b,g,I)  = { J <= I : Score(I, J) >= alpha * max_J' Score(I, J') }, ascending
+ * (the same q heads share each list, as tm_block_sparse_attn_fwd expects). The
+ * pooled keys and probe rows are bf16 and the scores fp32 (tensor cores), so
+ * a block whose score lies within rounding of the threshold may fall either
+ * way. alpha in [0, 1] (0 keeps every causal block); 1 <= probes and
+ * probes * (Hq / Hkv) <= 128; B * Hkv <= 65535.
+ * Memory (all DEVICE, caller-owned): workspace of at least
+ * tm_flashprefill_workspace_size bytes, 256-byte aligned; block_offsets of
+ * B * Hkv * nqb + 1 ints; block_indices of cap >= tm_flashprefill_index_capacity
+ * ints (the dense causal count, so a list never overflows); the number of
+ * entries written is block_offsets[B * Hkv * nqb]. scores_out (optional, may
+ * be NULL): B * Hkv * nqb * nqb floats receiving Score(I, J) at
+ * ((b * Hkv + g) * nqb + I) * nqb + J for J <= I. Asynchronous on `stream`
+ * (five launches, no host synchronisation).
+ */
+TM_API int tm_flashprefill_workspace_size(int B, int Hq, int Hkv, int N, int D, int probes,
+                                          long long* bytes);
+TM_API long long tm_flashprefill_index_capacity(int B, int Hkv, int N);
+TM_API int tm_flashprefill_block_index(const void* q, const void* k, int B, int Hq, int Hkv, int N,
+                                       int D, float scale, float alpha, int probes,
+                                       void* workspace, long long workspace_bytes,
+                                       int* block_offsets, int* block_indices, long long cap,
+                                       float* scores_out, void* stream);
+
+/*
  * Split schedule for the long q-blocks. The last L query rows of the triangle
  * (and the last rows of causal attention) see every earlier key, so one of
  * their items can cost more than a CTA's share of the launch when B * Hq is

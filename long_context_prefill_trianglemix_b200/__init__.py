@@ -28,7 +28,8 @@ EXPORTED = (
     "tm_debug_dump_tiles", "tm_debug_mma_probe", "tm_debug_schedule", "tm_get_device_status",
     "tm_status_string", "tm_attn_workspace_size", "tm_causal_attn_fwd_ws", "tm_triangle_attn_fwd_ws",
     "tm_trianglemix_attn_fwd_ws", "tm_trianglemix_attn_fwd_noalloc", "tm_block_sparse_attn_fwd",
-    "tm_trianglemix_sparse_attn_fwd",
+    "tm_trianglemix_sparse_attn_fwd", "tm_flashprefill_workspace_size",
+    "tm_flashprefill_index_capacity", "tm_flashprefill_block_index",
 )
 
 
@@ -78,6 +79,10 @@ def lib() -> ctypes.CDLL:
                                               vp]),
             "tm_trianglemix_sparse_attn_fwd": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci,
                                                     ci, ci, ci, vp, vp, cll, vp]),
+            "tm_flashprefill_workspace_size": (ci, [ci, ci, ci, ci, ci, ci, ctypes.POINTER(cll)]),
+            "tm_flashprefill_index_capacity": (cll, [ci, ci, ci]),
+            "tm_flashprefill_block_index": (ci, [vp, vp, ci, ci, ci, ci, ci, cf, cf, ci, vp, cll,
+                                                 vp, vp, cll, vp, vp]),
             "tm_get_device_status": (ci, [vp]),
             "tm_status_string": (ctypes.c_char_p, [ci]),
         }
@@ -177,6 +182,26 @@ def tm_trianglemix_sparse_attn_fwd(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L,
     return _check("tm_trianglemix_sparse_attn_fwd", lib().tm_trianglemix_sparse_attn_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, Hkv, N, D, scale, S, W, L, layer, tri_start,
         _ptr(block_offsets), _ptr(block_indices), int(nnz), _stream(stream)))
+
+
+def tm_flashprefill_workspace_size(B, Hq, Hkv, N, D, probes) -> int:
+    n = ctypes.c_longlong(0)
+    _check("tm_flashprefill_workspace_size", lib().tm_flashprefill_workspace_size(
+        B, Hq, Hkv, N, D, probes, ctypes.byref(n)))
+    return n.value
+
+
+def tm_flashprefill_index_capacity(B, Hkv, N) -> int:
+    return int(lib().tm_flashprefill_index_capacity(B, Hkv, N))
+
+
+def tm_flashprefill_block_index(q, k, B, Hq, Hkv, N, D, scale, alpha, probes, workspace,
+                                workspace_bytes, block_offsets, block_indices, cap,
+                                scores_out=None, stream=None):
+    return _check("tm_flashprefill_block_index", lib().tm_flashprefill_block_index(
+        _ptr(q), _ptr(k), B, Hq, Hkv, N, D, scale, alpha, probes, _ptr(workspace),
+        int(workspace_bytes), _ptr(block_offsets), _ptr(block_indices), int(cap),
+        _ptr(scores_out), _stream(stream)))
 
 
 def tm_attn_workspace_size(B, Hq, Hkv, N, D, causal, S, W, L, num_ctas=0) -> int:

@@ -183,6 +183,76 @@ TM_API int tm_trianglemix_sparse_attn_fwd(const void* q, const void* k, const vo
   return tm_triangle_attn_fwd(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L, stream);
 }
 
+namespace {
+
+int validate_discovery(const void* q, const void* k, int B, int Hq, int Hkv, int N, int D,
+                       float scale, float alpha, int probes) {
+  if (!q || !k || B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0) return TM_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return TM_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k)) return TM_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return TM_ERR_INVALID_ARG;
+  if (!std::isfinite(alpha) || alpha < 0.f || alpha > 1.f) return TM_ERR_INVALID_ARG;
+  if (probes < 1 || static_cast<long long>(probes) * (Hq / Hkv) > 128) return TM_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * Hkv > 65535) return TM_ERR_INVALID_ARG;
+  const long long rows = static_cast<long long>(B) * N;
+  if (rows > (1LL << 31) - 1 || static_cast<long long>(N) * Hq > (1LL << 31) - 1)
+    return TM_ERR_INVALID_ARG;
+  return TM_OK;
+}
+
+long long max_index_entries(int B, int Hkv, int N) {
+  const long long nqb = (N + TM_BLOCK_M - 1) / TM_BLOCK_M;
+  return static_cast<long long>(B) * Hkv * nqb * (nqb + 1) / 2;
+}
+
+}  // namespace
+
+TM_API int tm_flashprefill_workspace_size(int B, int Hq, int Hkv, int N, int D, int probes,
+                                          long long* bytes) {
+  if (!bytes) return TM_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0 || probes < 1 ||
+      static_cast<long long>(probes) * (Hq / Hkv) > 128)
+    return TM_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return TM_ERR_UNSUPPORTED;
+  *bytes = trimix::discovery_workspace_bytes(B, Hq, Hkv, N, D, probes);
+  return TM_OK;
+}
+
+TM_API long long tm_flashprefill_index_capacity(int B, int Hkv, int N) {
+  if (B < 1 || Hkv < 1 || N < 1) return -1;
+  return max_index_entries(B, Hkv, N);
+}
+
+TM_API int tm_flashprefill_block_index(const void* q, const void* k, int B, int Hq, int Hkv, int N,
+                                       int D, float scale, float alpha, int probes,
+                                       void* workspace, long long workspace_bytes,
+                                       int* block_offsets, int* block_indices, long long cap,
+                                       float* scores_out, void* stream) {
+  if (int rc = validate_discovery(q, k, B, Hq, Hkv, N, D, scale, alpha, probes)) return rc;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || !block_offsets ||
+      !block_indices || (reinterpret_cast<uintptr_t>(block_offsets) & 3u) ||
+      (reinterpret_cast<uintptr_t>(block_indices) & 3u) ||
+      (reinterpret_cast<uintptr_t>(scores_out) & 3u))
+    return TM_ERR_INVALID_ARG;
+  const long long need = max_index_entries(B, Hkv, N);
+  if (cap < need || need > (1LL << 31) - 1) return TM_ERR_INVALID_ARG;
+  if (workspace_bytes < trimix::discovery_workspace_bytes(B, Hq, Hkv, N, D, probes))
+    return TM_ERR_INVALID_ARG;
+  const long long rows = static_cast<long long>(B) * N;
+  if (overlaps(workspace, workspace_bytes, q, rows * Hq * D * 2) ||
+      overlaps(workspace, workspace_bytes, k, rows * Hkv * D * 2))
+    return TM_ERR_INVALID_ARG;
+  trimix::DiscArgs a;
+  a.q = q; a.k = k;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.N = N; a.D = D; a.P = probes;
+  a.scale = scale; a.alpha = alpha;
+  a.ws = workspace; a.ws_bytes = workspace_bytes;
+  a.offsets = block_offsets; a.indices = block_indices;
+  a.scores_out = scores_out;
+  a.stream = stream;
+  return trimix::launch_discovery(a);
+}
+
 TM_API int tm_attn_workspace_size(int B, int Hq, int Hkv, int N, int D, int causal, int S, int W,
                                   int L, int num_ctas, long long* bytes) {
   if (!bytes || B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0) return TM_ERR_INVALID_ARG;

@@ -96,7 +96,7 @@ constexpr long long kSplitOverheadTiles = 1;
 // Where a wait gave up (recorded with the timeout, for diagnosis).
 enum WaitSite : int {
   kSiteQEmpty = 1, kSiteKvEmpty, kSiteQFull, kSiteKvFull, kSiteOEmpty, kSitePFull,
-  kSiteSFull, kSiteOFull, kSiteProbe
+  kSiteSFull, kSiteOFull, kSiteProbe, kSiteDisc
 };
 
 template <int D>
@@ -1027,6 +1027,10 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
+// ------------------------------------------------------------------ pattern discovery
+
+#include "tm_discover.cuh"
+
 // ------------------------------------------------------------------ host side
 
 namespace {
@@ -1042,6 +1046,7 @@ struct DeviceInfo {
   int sms = 0;
   bool attr_set[2] = {false, false};
   bool probe_attr_set[2] = {false, false};
+  bool disc_attr_set[2] = {false, false};
 };
 
 std::mutex g_mutex;
@@ -1249,7 +1254,94 @@ int launch_attention_d(const LaunchArgs& a, DeviceInfo* di) {
   return cudaGetLastError() == cudaSuccess ? TM_OK : TM_ERR_CUDA;
 }
 
+// [planes, rows, D] bf16 (D contiguous), 64-column x 128-row boxes, 128-byte swizzle.
+int encode_3d(CUtensorMap* m, const void* base, int D, long long rows, long long planes) {
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)planes};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? TM_OK : TM_ERR_CUDA;
+}
+
+// Discovery workspace: pooled keys, probe rows, scores, counts (256-byte aligned).
+struct DiscLayout {
+  long long kbar, probes, scores, counts, total;
+};
+DiscLayout disc_layout(int B, int Hkv, int N, int D, int R) {
+  auto al = [](long long x) { return (x + 255) / 256 * 256; };
+  const long long lists = static_cast<long long>(B) * Hkv * ((N + BM - 1) / BM);
+  const long long nqb = (N + BM - 1) / BM;
+  DiscLayout l;
+  l.kbar = 0;
+  l.probes = l.kbar + al(lists * D * 2);
+  l.scores = l.probes + al(lists * R * D * 2);
+  l.counts = l.scores + al(lists * nqb * 4);
+  l.total = l.counts + al(lists * 4);
+  return l;
+}
+
+template <int D>
+int launch_discovery_d(const DiscArgs& a, DeviceInfo* di) {
+  const int kidx = D == 128 ? 1 : 0;
+  if (!di->disc_attr_set[kidx]) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (cudaFuncSetAttribute(score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DiscCfg<D>::kSmem) != cudaSuccess)
+      return TM_ERR_CUDA;
+    di->disc_attr_set[kidx] = true;
+  }
+  const int G = a.Hq / a.Hkv, R = G * a.P, nqb = (a.N + BM - 1) / BM;
+  const DiscLayout l = disc_layout(a.B, a.Hkv, a.N, D, R);
+  if (a.ws_bytes < l.total) return TM_ERR_INVALID_ARG;
+  uint8_t* ws = static_cast<uint8_t*>(a.ws);
+  DiscParams p;
+  p.B = a.B; p.Hkv = a.Hkv; p.N = a.N; p.G = G; p.nqb = nqb; p.P = a.P; p.R = R;
+  p.qbt = 128 / R;
+  p.sl2 = a.scale * 1.4426950408889634f;
+  p.alpha = a.alpha;
+  p.q = static_cast<const uint16_t*>(a.q);
+  p.k = static_cast<const uint16_t*>(a.k);
+  p.kbar = reinterpret_cast<uint16_t*>(ws + l.kbar);
+  p.probes = reinterpret_cast<uint16_t*>(ws + l.probes);
+  p.scores = a.scores_out ? a.scores_out : reinterpret_cast<float*>(ws + l.scores);
+  p.counts = reinterpret_cast<int*>(ws + l.counts);
+  p.offsets = a.offsets;
+  p.indices = a.indices;
+  const long long BH = static_cast<long long>(a.B) * a.Hkv;
+  CUtensorMap tp, tkb;
+  if (encode_3d(&tp, p.probes, D, static_cast<long long>(nqb) * R, BH) ||
+      encode_3d(&tkb, p.kbar, D, nqb, BH))
+    return TM_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(a.stream);
+  const dim3 g1(nqb, static_cast<unsigned>(BH));
+  pool_probe_kernel<D><<<g1, kDiscThreads, 0, st>>>(p);
+  const dim3 g2((nqb + p.qbt - 1) / p.qbt, static_cast<unsigned>(BH));
+  score_kernel<D><<<g2, kDiscThreads, DiscCfg<D>::kSmem, st>>>(tp, tkb, p);
+  const long long lists = BH * nqb;
+  const unsigned wblocks = static_cast<unsigned>((lists * 32 + 255) / 256);
+  count_kernel<<<wblocks, 256, 0, st>>>(p);
+  scan_kernel<<<1, 1024, 0, st>>>(p);
+  write_index_kernel<<<wblocks, 256, 0, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? TM_OK : TM_ERR_CUDA;
+}
+
 }  // namespace
+
+long long discovery_workspace_bytes(int B, int Hq, int Hkv, int N, int D, int P) {
+  return disc_layout(B, Hkv, N, D, (Hq / Hkv) * P).total;
+}
+
+int launch_discovery(const DiscArgs& a) {
+  DeviceInfo* di = nullptr;
+  if (int rc = device_info(&di)) return rc;
+  if (a.D == 128) return launch_discovery_d<128>(a, di);
+  if (a.D == 64) return launch_discovery_d<64>(a, di);
+  return TM_ERR_UNSUPPORTED;
+}
 
 int launch_attention(const LaunchArgs& a) {
   DeviceInfo* di = nullptr;

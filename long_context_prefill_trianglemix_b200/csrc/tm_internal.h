@@ -27,12 +27,27 @@ struct LaunchArgs {
   void* stream;
 };
 
+struct DiscArgs {
+  const void* q;
+  const void* k;
+  int B, Hq, Hkv, N, D, P;
+  float scale, alpha;
+  void* ws;
+  long long ws_bytes;
+  int* offsets;
+  int* indices;
+  float* scores_out;  // optional: the block scores land here instead of the workspace
+  void* stream;
+};
+
 // All return a tm_status value.
 int launch_attention(const LaunchArgs& a);
 int launch_dump_tiles(const Pattern& p, int* out_dev, long long cap, void* stream);
 int launch_mma_probe(const void* q, const void* k, const void* v, float* s_out, float* o_out,
                      int D, void* stream);
 int read_and_clear_device_status(void* stream);
+int launch_discovery(const DiscArgs& a);
+long long discovery_workspace_bytes(int B, int Hq, int Hkv, int N, int D, int P);
 int debug_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ctas, int split,
                    int* out, long long cap, long long* count);
 // Workspace bytes the split schedule needs on num_ctas CTAs (<= 0: the

@@ -15,6 +15,15 @@ them. The value recipe per workload:
             multiplied by 8 in k[..., g, :] and in every q head of g's group
             (the same channels in q and k, so they raise the logits).
 * headscale: q and k heads each get their own factor ~ U[0.5, 2].
+* planted:  as plain, then attention structure of the kind block-sparse
+            methods find (FlashPrefill summary, section 2.1: vertical, slash
+            and block patterns) is planted in the last channels of q and k:
+            four sine/cosine channel pairs of position with long periods
+            (8192 .. 65536 tokens), equal in q and k, so that q_i . k_j gains
+            a sum of cos(w (i - j)) terms that favours nearby keys; and, per kv
+            head, 16 seeded key blocks whose keys gain +3 in one more channel
+            that every query of the group also carries (+3), so every later
+            query attends to them.
 
 Element values come from the C generator in ``tm_inputs.c`` (splitmix64 +
 Box-Muller, bf16 round-to-nearest-even). Channel choices and head factors are
@@ -149,6 +158,11 @@ WORKLOADS = {
     # fraction of the launch and is cut into pieces when a workspace is given.
     "llama3-8b-128k-tp8": Workload("llama3-8b-128k-tp8", B=1, Hq=4, Hkv=1, N=131072, D=128,
                                    S=64, W=2048, L=256, layers=2, tri_start=1),
+    # The 128K Llama-3-8B shape with planted vertical and local attention
+    # structure, the input of block pattern discovery.
+    "llama3-8b-128k-planted": Workload("llama3-8b-128k-planted", B=1, Hq=32, Hkv=8, N=131072,
+                                       D=128, S=64, W=2048, L=256, layers=2, tri_start=1,
+                                       recipe="planted"),
     "qwen2.5-7b-128k-tp4": Workload("qwen2.5-7b-128k-tp4", B=1, Hq=7, Hkv=1, N=131072, D=128,
                                     S=64, W=1024, L=128, layers=28, tri_start=20,
                                     recipe="headscale"),
@@ -188,9 +202,48 @@ def scales_for(wl: Workload, layer: int = 0):
                 ck[g, c] = 8.0
                 cq[g * G:(g + 1) * G, c] = 8.0
         return (None, cq.reshape(-1)), (None, ck.reshape(-1)), none
+    if wl.recipe == "planted":
+        return none, none, none
     if wl.recipe == "headscale":
         return (head_scales(seed, wl.Hq, 2000), None), (head_scales(seed, wl.Hkv, 2001), None), none
     raise ValueError(wl.recipe)
+
+
+PLANT_PERIODS = (8192.0, 16384.0, 32768.0, 65536.0)
+PLANT_AMP = 2.0
+PLANT_VERTICAL_BLOCKS = 16
+PLANT_VERTICAL_AMP = 3.0
+
+
+def planted_vertical_blocks(seed: int, Hkv: int, nblocks: int):
+    """Per kv head, the seeded key blocks of the planted recipe's vertical pattern."""
+    return [sorted({int(_uniform(seed, 4000 + g, n) * nblocks)
+                    for n in range(PLANT_VERTICAL_BLOCKS)}) for g in range(Hkv)]
+
+
+def _plant(arr: np.ndarray, tensor_id: int, seed: int, G: int, BM: int = 128):
+    """Add the planted structure to bf16 bits arr [B, N, H, D] in place (last
+    2 * len(PLANT_PERIODS) + 1 channels; float32 sums rounded to bf16 RNE).
+    Uses torch's CPU tensors only for their fast strided copies."""
+    import torch
+    B, N, H, D = arr.shape
+    nc = 2 * len(PLANT_PERIODS) + 1
+    sl = torch.from_numpy(arr.view(np.int16))[..., D - nc:]
+    x = ((sl.to(torch.int32) & 0xFFFF) << 16).view(torch.float32)      # [B, N, H, nc]
+    pos = np.arange(N, dtype=np.float64)
+    add = np.zeros((N, nc), np.float32)
+    for c, period in enumerate(PLANT_PERIODS):
+        w = 2.0 * np.pi / period
+        add[:, nc - 1 - 2 * c] = PLANT_AMP * np.cos(w * pos)           # channel D - 1 - 2c
+        add[:, nc - 2 - 2 * c] = PLANT_AMP * np.sin(w * pos)           # channel D - 2 - 2c
+    x += torch.from_numpy(add)[None, :, None, :]
+    if tensor_id == TENSOR_Q:
+        x[..., 0] += PLANT_VERTICAL_AMP                                 # channel D - nc
+    elif tensor_id == TENSOR_K:
+        for g, blocks in enumerate(planted_vertical_blocks(seed, H, (N + BM - 1) // BM)):
+            for blk in blocks:
+                x[:, blk * BM:(blk + 1) * BM, g, 0] += PLANT_VERTICAL_AMP
+    sl.copy_(x.to(torch.bfloat16).view(torch.int16))
 
 
 def make_qkv(wl: Workload, layer: int = 0, out=None, N: int | None = None, nthreads=None):
@@ -208,6 +261,8 @@ def make_qkv(wl: Workload, layer: int = 0, out=None, N: int | None = None, nthre
     for arr, shp, tid, hs, cs in zip(out, shapes, (TENSOR_Q, TENSOR_K, TENSOR_V),
                                     (qh, kh, vh), (qc, kc, vc)):
         fill_bf16(arr.reshape(-1), *shp[:2], shp[2], shp[3], seed, tid, hs, cs, nthreads)
+        if wl.recipe == "planted" and tid != TENSOR_V:
+            _plant(arr.reshape(shp), tid, seed, wl.Hq // wl.Hkv)
     return out
 
 
@@ -216,12 +271,15 @@ def bf16_bits_to_f32(a: np.ndarray) -> np.ndarray:
 
 
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
-    """Round-to-nearest-even float32 -> bf16 bits (NaN kept quiet)."""
-    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    nan = (u & 0x7F800000) == 0x7F800000
-    nan &= (u & 0x007FFFFF) != 0
-    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
-    r[nan] = ((u[nan] >> 16) | 0x40).astype(np.uint16)
+    """Round-to-nearest-even float32 -> bf16 bits (NaN kept quiet). The 32-bit
+    sum can wrap only for NaN bit patterns, which are handled separately."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+    r = ((u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16))
+    r = r.astype(np.uint16)
+    nan = (u & np.uint32(0x7F800000)) == np.uint32(0x7F800000)
+    nan &= (u & np.uint32(0x007FFFFF)) != 0
+    if nan.any():
+        r[nan] = ((u[nan] >> np.uint32(16)) | np.uint32(0x40)).astype(np.uint16)
     return r
 
 

@@ -48,6 +48,9 @@ def _load():
         lib.oracle_block_sparse_attention.argtypes = [
             vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_dbl, c_int, c_int, vp, vp, c_ll, vp,
             c_ll, vp, c_int]
+        lib.oracle_flashprefill_scores.restype = c_int
+        lib.oracle_flashprefill_scores.argtypes = [vp, vp, c_int, c_int, c_int, c_int, c_int,
+                                                   c_dbl, c_int, c_int, vp, c_int]
         for name in ("oracle_tile_list_bruteforce", "oracle_tile_list_rows"):
             f = getattr(lib, name)
             f.restype = c_int
@@ -157,3 +160,32 @@ def block_sparse_attention(q, k, v, B, Hq, Hkv, N, D, scale, offsets, indices, r
     if rc != 0:
         raise ValueError("oracle_block_sparse_attention: bad argument")
     return out
+
+
+def flashprefill_scores(q, k, B, Hq, Hkv, N, D, scale, probes, BS=128, nthreads=None):
+    """fp64 block scores Score(I, J) [B * Hkv, nqb, nqb] of the discovery step."""
+    lib = _load()
+    for a in (q, k):
+        assert a.dtype == np.uint16 and a.flags.c_contiguous
+    nb = (N + BS - 1) // BS
+    out = np.zeros((B * Hkv, nb, nb), np.float64)
+    rc = lib.oracle_flashprefill_scores(q.ctypes.data, k.ctypes.data, B, Hq, Hkv, N, D,
+                                        float(scale), probes, BS, out.ctypes.data,
+                                        nthreads or hardware_threads())
+    if rc != 0:
+        raise ValueError("oracle_flashprefill_scores: bad argument")
+    return out
+
+
+def flashprefill_select(scores, alpha):
+    """Kept blocks per list from the scores: J <= I with Score >= alpha * max_J Score.
+    Returns (offsets int32 [n_lists + 1], indices int32)."""
+    BH, nb, _ = scores.shape
+    lists = []
+    for bg in range(BH):
+        for I in range(nb):
+            row = scores[bg, I, :I + 1]
+            lists.append(np.flatnonzero(row >= alpha * row.max()).astype(np.int32))
+    off = np.zeros(len(lists) + 1, np.int32)
+    off[1:] = np.cumsum([len(x) for x in lists])
+    return off, (np.concatenate(lists) if lists else np.zeros(0, np.int32))

@@ -32,7 +32,9 @@
 //   * causal and masked rows match a library softmax-attention routine;
 //   * block-sparse: every causal block listed gives causal attention exactly;
 //     q = 0 gives the mean of v over the kept keys; rows match the library
-//     routine under a block mask built independently; empty lists give 0.
+//     routine under a block mask built independently; empty lists give 0;
+//   * discovery scores: q = 0 gives 1 / (I + 1); one probe on one head gives
+//     a plain softmax (a worked example with closed-form values).
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
@@ -290,6 +292,65 @@ int oracle_block_sparse_attention(const uint16_t* q, const uint16_t* k, const ui
           for (int d = 0; d < D; ++d) op[d] = o[size_t(d)] / l;
         }
       }
+    }
+  });
+  return 0;
+}
+
+// Block pattern discovery (FlashPrefill summary, section 2.1: probe queries
+// spread evenly over each query block, keys average-pooled per block;
+// section 2.2: keep the key blocks whose score reaches alpha times the best
+// score of the query block). In fp64, step by step, for batch b, kv head g
+// and query block I with rows [r0, r1):
+//   kbar_J      = mean of k[b, j, g, :] over the keys j of block J
+//   probe rows  max(r0, r0 + ((p + 1) (r1 - r0)) / P - 1), p = 0 .. P-1, in each
+//               q head h of g's group (a block shorter than P repeats rows)
+//   pi_{h,p}(J) = softmax over J in [0, I] of scale * q[b, row, h, :] . kbar_J
+//   Score(I, J) = mean over (h, p) of pi_{h,p}(J)
+// scores: [B * Hkv, nqb, nqb] (J > I left 0). Block size BS for both queries
+// and keys. Returns 0, or -1 on a bad argument.
+int oracle_flashprefill_scores(const uint16_t* q, const uint16_t* k, int B, int Hq, int Hkv, int N,
+                               int D, double scale, int P, int BS, double* scores, int nthreads) {
+  if (!q || !k || !scores || B < 1 || Hq < 1 || Hkv < 1 || N < 1 || D < 1 || Hq % Hkv != 0 ||
+      P < 1 || BS < 1)
+    return -1;
+  const int G = Hq / Hkv;
+  const long long nb = (N + BS - 1) / BS;
+  std::vector<double> kbar(size_t(B) * Hkv * nb * D, 0.0);
+  for (long long b = 0; b < B; ++b)
+    for (int g = 0; g < Hkv; ++g)
+      for (long long J = 0; J < nb; ++J) {
+        const long long j0 = J * BS, j1 = std::min<long long>(N, j0 + BS);
+        double* kb = &kbar[size_t(((b * Hkv + g) * nb + J) * D)];
+        for (long long j = j0; j < j1; ++j)
+          for (int d = 0; d < D; ++d) kb[d] += bf16_to_double(k[((b * N + j) * Hkv + g) * D + d]);
+        for (int d = 0; d < D; ++d) kb[d] /= double(j1 - j0);
+      }
+  parallel_for((long long)B * Hkv * nb, nthreads, [&](long long ub, long long ue) {
+    std::vector<double> logit, mean;
+    for (long long u = ub; u < ue; ++u) {
+      const long long bg = u / nb, I = u % nb, b = bg / Hkv, g = bg % Hkv;
+      const long long r0 = I * BS, r1 = std::min<long long>(N, r0 + BS);
+      logit.assign(size_t(I + 1), 0.0);
+      mean.assign(size_t(I + 1), 0.0);
+      for (int h = 0; h < G; ++h)
+        for (int pi = 0; pi < P; ++pi) {
+          const long long row = std::max(r0, r0 + ((pi + 1) * (r1 - r0)) / P - 1);
+          const uint16_t* qp = q + ((b * N + row) * Hq + g * G + h) * (long long)D;
+          double mx = -std::numeric_limits<double>::infinity();
+          for (long long J = 0; J <= I; ++J) {
+            const double* kb = &kbar[size_t((bg * nb + J) * D)];
+            double acc = 0.0;
+            for (int d = 0; d < D; ++d) acc += bf16_to_double(qp[d]) * kb[d];
+            logit[size_t(J)] = scale * acc;
+            mx = std::max(mx, logit[size_t(J)]);
+          }
+          double z = 0.0;
+          for (long long J = 0; J <= I; ++J) z += std::exp(logit[size_t(J)] - mx);
+          for (long long J = 0; J <= I; ++J) mean[size_t(J)] += std::exp(logit[size_t(J)] - mx) / z;
+        }
+      double* out = scores + (bg * nb + I) * nb;
+      for (long long J = 0; J < nb; ++J) out[J] = J <= I ? mean[size_t(J)] / double(G * P) : 0.0;
     }
   });
   return 0;

@@ -1,0 +1,172 @@
+"""Parity of block pattern discovery (tm_flashprefill_block_index, through the
+C ABI) with the fp64 oracle. The scores are compared value by value; the
+kept lists are compared where the decision is unique: every block whose
+oracle score clears the threshold by a margin must be listed, every block
+below it by the margin must not, and blocks within the margin (where bf16
+pooled keys and fp32 scores may tip the comparison) may go either way. The
+discovered index then drives block-sparse attention, checked against the
+oracle on the lists where both indices agree.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import long_context_prefill_trianglemix_b200 as tm
+from long_context_prefill_trianglemix_b200 import inputs as I
+from gpu_util import assert_close, from_dev, to_dev
+
+pytestmark = pytest.mark.gpu
+
+MARGIN = 2e-2  # relative band around the threshold where either decision is accepted
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_ready():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from long_context_prefill_trianglemix_b200 import build
+    build.build_lib()
+    yield
+    assert tm.tm_get_device_status() == tm.TM_OK
+
+
+def rand_bits(shape, seed, scale=1.0):
+    g = np.random.default_rng(seed)
+    return I.f32_to_bf16_bits((g.standard_normal(shape) * scale).astype(np.float32))
+
+
+def discover(dq, dk, B, Hq, Hkv, N, D, scale, alpha, probes, with_scores=True):
+    import torch
+    nqb = (N + 127) // 128
+    ws_n = tm.tm_flashprefill_workspace_size(B, Hq, Hkv, N, D, probes)
+    ws = torch.empty(ws_n, dtype=torch.uint8, device="cuda")
+    cap = tm.tm_flashprefill_index_capacity(B, Hkv, N)
+    off = torch.full((B * Hkv * nqb + 1,), -1, dtype=torch.int32, device="cuda")
+    idx = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
+    sc = (torch.zeros(B * Hkv * nqb * nqb, dtype=torch.float32, device="cuda")
+          if with_scores else None)
+    tm.tm_flashprefill_block_index(dq, dk, B, Hq, Hkv, N, D, scale, alpha, probes, ws, ws_n, off,
+                                   idx, cap, sc)
+    torch.cuda.synchronize()
+    assert tm.tm_get_device_status() == tm.TM_OK
+    o = off.cpu().numpy()
+    return o, idx.cpu().numpy()[: o[-1]], (None if sc is None else
+                                           sc.cpu().numpy().reshape(B * Hkv, nqb, nqb)), (off, idx)
+
+
+def check_lists(off, idx, ref_scores, alpha):
+    BH, nb, _ = ref_scores.shape
+    assert off[0] == 0 and (np.diff(off) >= 0).all()
+    n_free, agree = 0, np.zeros(BH * nb, bool)
+    ref_off, ref_idx = oracle.flashprefill_select(ref_scores, alpha)
+    for r in range(BH * nb):
+        Ib = r % nb
+        row = ref_scores[r // nb, Ib, :Ib + 1]
+        th = alpha * row.max()
+        got = idx[off[r]:off[r + 1]]
+        assert (np.diff(got) > 0).all() and (got >= 0).all() and (got <= Ib).all(), (r, got)
+        s = set(got.tolist())
+        must = set(np.flatnonzero(row >= th * (1 + MARGIN)).tolist())
+        never = set(np.flatnonzero(row < th * (1 - MARGIN)).tolist())
+        assert must <= s, (r, sorted(must - s))
+        assert not (s & never), (r, sorted(s & never))
+        n_free += Ib + 1 - len(must) - len(never)
+        agree[r] = s == set(ref_idx[ref_off[r]:ref_off[r + 1]].tolist())
+    return n_free, agree
+
+
+CASES = [  # B, Hq, Hkv, N, D, probes, alpha, scale of q/k
+    (1, 4, 1, 4096, 128, 4, 0.5, 3.0),
+    (2, 8, 2, 3000, 64, 8, 0.3, 3.0),
+    (1, 7, 1, 2049, 128, 4, 0.7, 4.0),
+    (1, 2, 2, 300, 128, 16, 0.0, 1.0),
+    (1, 32, 8, 16384, 128, 4, 0.5, 3.0),
+    (1, 1, 1, 40000, 128, 1, 0.9, 4.0),
+    (1, 2, 1, 130, 64, 8, 0.5, 2.0),          # last block of 2 rows, 8 probes
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,D,probes,alpha,amp", CASES)
+def test_scores_and_lists_match_oracle(B, Hq, Hkv, N, D, probes, alpha, amp):
+    q = rand_bits((B, N, Hq, D), 71, amp)
+    k = rand_bits((B, N, Hkv, D), 72, amp)
+    scale = 1.0 / math.sqrt(D)
+    off, idx, sc, _ = discover(to_dev(q), to_dev(k), B, Hq, Hkv, N, D, scale, alpha, probes)
+    ref = oracle.flashprefill_scores(q, k, B, Hq, Hkv, N, D, scale, probes)
+    nb = ref.shape[1]
+    tri = np.tril(np.ones((nb, nb), bool))
+    np.testing.assert_allclose(sc[:, tri], ref[:, tri], rtol=2e-2, atol=1e-5)
+    n_free, agree = check_lists(off, idx, ref, alpha)
+    assert agree.mean() > 0.9, agree.mean()
+
+
+def test_discovered_index_drives_block_sparse_attention():
+    import torch
+    B, Hq, Hkv, N, D, probes, alpha = 1, 8, 2, 8192, 128, 4, 0.5
+    q, k, v = (rand_bits((B, N, h, D), s, a) for h, s, a in ((Hq, 81, 3.0), (Hkv, 82, 3.0),
+                                                               (Hkv, 83, 1.0)))
+    scale = 1.0 / math.sqrt(D)
+    dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
+    off, idx, _, (doff, didx) = discover(dq, dk, B, Hq, Hkv, N, D, scale, alpha, probes, False)
+    o = torch.empty_like(dq)
+    tm.tm_block_sparse_attn_fwd(dq, dk, dv, o, B, Hq, Hkv, N, D, scale, doff, didx, len(idx))
+    torch.cuda.synchronize()
+    ref_scores = oracle.flashprefill_scores(q, k, B, Hq, Hkv, N, D, scale, probes)
+    _, agree = check_lists(off, idx, ref_scores, alpha)
+    ref_off, ref_idx = oracle.flashprefill_select(ref_scores, alpha)
+    want = oracle.block_sparse_attention(q, k, v, B, Hq, Hkv, N, D, scale, ref_off, ref_idx)
+    got = from_dev(o)
+    nqb = (N + 127) // 128
+    G = Hq // Hkv
+    rows = [(r // nqb, r % nqb) for r in np.flatnonzero(agree)]  # (kv head, q-block); B = 1
+    assert len(rows) > 0.9 * Hkv * nqb
+    sel_g = np.concatenate([got[0, qb * 128:(qb + 1) * 128, g * G:(g + 1) * G] for g, qb in rows])
+    sel_w = np.concatenate([want[0, qb * 128:(qb + 1) * 128, g * G:(g + 1) * G] for g, qb in rows])
+    assert_close(sel_g, sel_w, "attention over the discovered index")
+    density = len(idx) / (Hkv * nqb * (nqb + 1) / 2)
+    assert 0.0 < density < 1.0
+
+
+def test_argument_errors():
+    import torch
+    B, Hq, Hkv, N, D = 1, 4, 1, 1024, 128
+    dq = torch.zeros((B, N, Hq, D), dtype=torch.bfloat16, device="cuda")
+    dk = torch.zeros((B, N, Hkv, D), dtype=torch.bfloat16, device="cuda")
+    ws_n = tm.tm_flashprefill_workspace_size(B, Hq, Hkv, N, D, 4)
+    ws = torch.empty(ws_n, dtype=torch.uint8, device="cuda")
+    cap = tm.tm_flashprefill_index_capacity(B, Hkv, N)
+    off = torch.empty(B * Hkv * 8 + 1, dtype=torch.int32, device="cuda")
+    idx = torch.empty(cap, dtype=torch.int32, device="cuda")
+    L = tm.lib()
+    base = (dq.data_ptr(), dk.data_ptr(), B, Hq, Hkv, N, D, 0.1)
+    assert L.tm_flashprefill_block_index(*base, 1.5, 4, ws.data_ptr(), ws_n, off.data_ptr(),
+                                         idx.data_ptr(), cap, None, None) == tm.TM_ERR_INVALID_ARG
+    assert L.tm_flashprefill_block_index(*base, 0.5, 33, ws.data_ptr(), ws_n, off.data_ptr(),
+                                         idx.data_ptr(), cap, None, None) == tm.TM_ERR_INVALID_ARG
+    assert L.tm_flashprefill_block_index(*base, 0.5, 4, ws.data_ptr(), ws_n - 1, off.data_ptr(),
+                                         idx.data_ptr(), cap, None, None) == tm.TM_ERR_INVALID_ARG
+    assert L.tm_flashprefill_block_index(*base, 0.5, 4, ws.data_ptr(), ws_n, off.data_ptr(),
+                                         idx.data_ptr(), cap - 1, None, None) == tm.TM_ERR_INVALID_ARG
+
+
+def test_planted_32k_structure_is_found():
+    """Llama-3-8B shape at 32K with planted local and vertical structure: every
+    list checked against the oracle's scores (unique decisions), a sparse
+    result, and the planted vertical blocks kept by most later query blocks."""
+    import dataclasses
+    wl = dataclasses.replace(I.WORKLOADS["llama3-8b-128k-planted"], N=32768)
+    q, k, v = I.make_qkv(wl)
+    alpha, probes = 0.3, 4
+    off, idx, sc, _ = discover(to_dev(q), to_dev(k), wl.B, wl.Hq, wl.Hkv, wl.N, wl.D, wl.scale,
+                               alpha, probes)
+    ref = oracle.flashprefill_scores(q, k, wl.B, wl.Hq, wl.Hkv, wl.N, wl.D, wl.scale, probes)
+    nb = ref.shape[1]
+    tri = np.tril(np.ones((nb, nb), bool))
+    np.testing.assert_allclose(sc[:, tri], ref[:, tri], rtol=2e-2, atol=1e-5)
+    _, agree = check_lists(off, idx, ref, alpha)
+    assert agree.mean() > 0.9
+    density = len(idx) / (wl.Hkv * nb * (nb + 1) / 2)
+    assert 0.02 < density < 0.5, density

@@ -52,3 +52,35 @@ def test_headscale_recipe_range():
     (qh, _), (kh, _), _ = I.scales_for(wl)
     assert qh.shape == (28,) and kh.shape == (4,)
     assert (qh >= 0.5).all() and (qh <= 2.0).all() and len(set(qh.tolist())) == 28
+
+
+def test_planted_recipe_adds_exactly_its_structure():
+    import dataclasses
+    base = I.WORKLOADS["llama3-8b-128k-planted"]
+    wl = dataclasses.replace(base, N=1000, Hq=4, Hkv=2)
+    plain = dataclasses.replace(wl, recipe="plain")
+    q, k, v = I.make_qkv(wl)
+    q0, k0, v0 = I.make_qkv(plain)
+    D, nc = wl.D, 2 * len(I.PLANT_PERIODS) + 1
+    assert np.array_equal(v, v0)
+    assert np.array_equal(q[..., :D - nc], q0[..., :D - nc])
+    assert np.array_equal(k[..., :D - nc], k0[..., :D - nc])
+    pos = np.arange(wl.N)
+    for c, period in enumerate(I.PLANT_PERIODS):
+        w = 2 * np.pi / period
+        for ch, val in ((D - 1 - 2 * c, np.cos(w * pos)), (D - 2 - 2 * c, np.sin(w * pos))):
+            for a, a0 in ((q, q0), (k, k0)):
+                want = I.bf16_bits_to_f32(a0[..., ch]) + np.float32(I.PLANT_AMP) * \
+                    val.astype(np.float32)[None, :, None]
+                assert np.array_equal(a[..., ch], I.f32_to_bf16_bits(want.astype(np.float32)))
+    ch = D - nc
+    dq = I.bf16_bits_to_f32(q[..., ch]) - I.bf16_bits_to_f32(q0[..., ch])
+    assert np.allclose(dq, I.PLANT_VERTICAL_AMP, atol=0.05)
+    blocks = I.planted_vertical_blocks(0, wl.Hkv, (wl.N + 127) // 128)
+    dk = I.bf16_bits_to_f32(k[..., ch]) - I.bf16_bits_to_f32(k0[..., ch])
+    for g in range(wl.Hkv):
+        in_v = np.zeros(wl.N, bool)
+        for b in blocks[g]:
+            in_v[b * 128:(b + 1) * 128] = True
+        assert np.allclose(dk[0, in_v, g], I.PLANT_VERTICAL_AMP, atol=0.05)
+        assert np.array_equal(dk[0, ~in_v, g], np.zeros((~in_v).sum(), np.float32))
