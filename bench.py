@@ -314,6 +314,29 @@ def run_ours(args):
     bs_ms = sum(bs_ev[s][0].elapsed_time(bs_ev[s][1]) for s in range(args.steps))
     bs_f = float(len(bs_idx)) * (wl.Hq // wl.Hkv) * 4.0 * BM * BN * wl.D
 
+    # per-head bands (seeded windows 512..4096 and sinks {0, 64} per q head) on the
+    # same inputs, timed on its own; useful FLOPs count each head's own tiles
+    hS, hW = I.head_bands(wl.Hq, 0)
+    head_tiles = sum(tm.tm_kept_tiles(wl.N, False, int(hS[h]), int(hW[h]), wl.L)
+                     for h in range(wl.Hq)) * wl.B
+    hb_ws_n = tm.tm_attn_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.N, wl.D, False, int(hS.max()),
+                                        int(hW.max()), wl.L)
+    hb_ws = torch.empty(max(hb_ws_n, 16), dtype=torch.uint8, device="cuda")
+
+    def heads_call():
+        tm.tm_triangle_attn_fwd_heads(dq, dk, dv, do, wl.B, wl.Hq, wl.Hkv, wl.N, wl.D, wl.scale,
+                                      hS, hW, wl.L, hb_ws, hb_ws_n, stream)
+
+    for _ in range(args.warmup):
+        heads_call()
+    hb_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for s in range(args.steps):
+        hb_ev[s][0].record(stream)
+        heads_call()
+        hb_ev[s][1].record(stream)
+    torch.cuda.synchronize()
+    hb_ms = sum(hb_ev[s][0].elapsed_time(hb_ev[s][1]) for s in range(args.steps))
+
     # block pattern discovery (probes per block, alpha) producing an index on the
     # GPU, then block-sparse attention over it; both timed on their own. Seeded
     # N(0,1) tensors have no attention structure to find, so this leg runs on the
@@ -355,8 +378,8 @@ def run_ours(args):
     dsa_ms = sum(dv_ev[s][1].elapsed_time(dv_ev[s][2]) for s in range(args.steps))
     f_nnz = int(f_off[-1].item())
 
-    total_ms, tri_sum, e2e_ms, bs_ms, disc_ms, dsa_ms = reduce_over_ranks(
-        [total_ms, tri_sum, e2e_ms, bs_ms, disc_ms, dsa_ms], device="cuda")
+    total_ms, tri_sum, e2e_ms, bs_ms, disc_ms, dsa_ms, hb_ms = reduce_over_ranks(
+        [total_ms, tri_sum, e2e_ms, bs_ms, disc_ms, dsa_ms, hb_ms], device="cuda")
 
     peaks = load_peaks()
     tri_avg = tri_sum / args.steps
@@ -399,6 +422,15 @@ def run_ours(args):
             "density_vs_causal": len(bs_idx) / (wl.B * wl.Hkv * ((wl.N + BM - 1) // BM)
                                                 * ((wl.N + BM - 1) // BM + 1) / 2),
             "speedup_vs_causal": (sum(cau_ms) / args.steps) / (bs_ms / args.steps),
+        },
+        "head_bands": {
+            "what": "tm_triangle_attn_fwd_heads, seeded per-head windows 512..4096 (log-uniform) "
+                    "and sinks {0, 64}, L shared; heads paired in band order",
+            "ms": hb_ms / args.steps,
+            "tflops_own_tiles": head_tiles * 4.0 * BM * BN * wl.D / (hb_ms / args.steps * 1e-3)
+                                / 1e12,
+            "own_tiles": int(head_tiles),
+            "speedup_vs_causal": (sum(cau_ms) / args.steps) / (hb_ms / args.steps),
         },
         "discovery": {
             "what": "tm_flashprefill_block_index (pooled keys, %d probe rows per block and q "

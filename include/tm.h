@@ -94,6 +94,26 @@ TM_API int tm_trianglemix_attn_fwd(const void* q, const void* k, const void* v, 
                                    int L, int layer, int tri_start, void* stream);
 
 /*
+ * Triangle attention with a band per q head: head h keeps the sinks j < S_h
+ * and the window i - j < W_h, all heads share the last-L rows. This is the
+ * bf16 reading of TriAttention's per-head regions (arXiv 2611.07256 abstract
+ * on the TriAttention page: each head's computed region is encoded by two
+ * diagonal-distance boundaries, independent of the context length); with both
+ * precision regions computed in bf16 the computed region is one band below
+ * the diagonal, here widened by the head's sinks.
+ * S_heads, W_heads: HOST arrays of Hq ints (S_h >= 0, W_h >= 1; S_h and W_h
+ * larger than N act as N); Hq <= 128. The heads of a kv group are paired in
+ * band order and a pair visits the union of its two bands (masked per head),
+ * so heads with similar bands cost nothing extra. workspace / workspace_bytes
+ * as for tm_triangle_attn_fwd_ws, sized by tm_attn_workspace_size with
+ * S = max S_h and W = max W_h (NULL and 0 split nothing).
+ */
+TM_API int tm_triangle_attn_fwd_heads(const void* q, const void* k, const void* v, void* o, int B,
+                                      int Hq, int Hkv, int N, int D, float scale,
+                                      const int* S_heads, const int* W_heads, int L,
+                                      void* workspace, long long workspace_bytes, void* stream);
+
+/*
  * Block-sparse causal attention from a caller's block index, on the same
  * kernels: the visited tiles of each q-block come from the index instead of a
  * closed form, the way the FlashPrefill summary (section 2.3) jumps straight
@@ -270,8 +290,9 @@ TM_API int tm_debug_mma_probe(const void* q, const void* k, const void* v, float
 
 /*
  * Host export of the persistent work split the kernels use on a grid of
- * num_ctas CTAs (the SM count on a B200); split != 0 gives the split schedule
- * of the *_ws calls, 0 the one of the calls without workspace. One record of
+ * num_ctas CTAs (the SM count on a B200). split: bit 0 gives the split
+ * schedule of the *_ws calls (else the one of the calls without workspace),
+ * bit 1 the pair rotation of per-head band launches. One record of
  * seven ints per work item, (cta, item, q-block, first q head
  * (batch * Hq + head), number of Q tiles 1 or 2, first tile, end tile), in the
  * order each CTA processes them; the tiles are positions [first, end) in the

@@ -29,7 +29,7 @@ EXPORTED = (
     "tm_status_string", "tm_attn_workspace_size", "tm_causal_attn_fwd_ws", "tm_triangle_attn_fwd_ws",
     "tm_trianglemix_attn_fwd_ws", "tm_trianglemix_attn_fwd_noalloc", "tm_block_sparse_attn_fwd",
     "tm_trianglemix_sparse_attn_fwd", "tm_flashprefill_workspace_size",
-    "tm_flashprefill_index_capacity", "tm_flashprefill_block_index",
+    "tm_flashprefill_index_capacity", "tm_flashprefill_block_index", "tm_triangle_attn_fwd_heads",
 )
 
 
@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
             "tm_trianglemix_sparse_attn_fwd": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci,
                                                     ci, ci, ci, vp, vp, cll, vp]),
             "tm_flashprefill_workspace_size": (ci, [ci, ci, ci, ci, ci, ci, ctypes.POINTER(cll)]),
+            "tm_triangle_attn_fwd_heads": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp, vp, ci,
+                                                vp, cll, vp]),
             "tm_flashprefill_index_capacity": (cll, [ci, ci, ci]),
             "tm_flashprefill_block_index": (ci, [vp, vp, ci, ci, ci, ci, ci, cf, cf, ci, vp, cll,
                                                  vp, vp, cll, vp, vp]),
@@ -184,6 +186,17 @@ def tm_trianglemix_sparse_attn_fwd(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L,
         _ptr(block_offsets), _ptr(block_indices), int(nnz), _stream(stream)))
 
 
+def tm_triangle_attn_fwd_heads(q, k, v, o, B, Hq, Hkv, N, D, scale, S_heads, W_heads, L,
+                               workspace=None, workspace_bytes=0, stream=None):
+    """Triangle attention with per-head sinks and windows (host int sequences of Hq)."""
+    Sh = np.ascontiguousarray(S_heads, dtype=np.int32)
+    Wh = np.ascontiguousarray(W_heads, dtype=np.int32)
+    assert Sh.size == Hq and Wh.size == Hq
+    return _check("tm_triangle_attn_fwd_heads", lib().tm_triangle_attn_fwd_heads(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, Hkv, N, D, scale, Sh.ctypes.data,
+        Wh.ctypes.data, L, _ptr(workspace), int(workspace_bytes), _stream(stream)))
+
+
 def tm_flashprefill_workspace_size(B, Hq, Hkv, N, D, probes) -> int:
     n = ctypes.c_longlong(0)
     _check("tm_flashprefill_workspace_size", lib().tm_flashprefill_workspace_size(
@@ -253,9 +266,11 @@ def tm_debug_mma_probe(q, k, v, s_out, o_out, D, stream=None):
         _ptr(q), _ptr(k), _ptr(v), _ptr(s_out), _ptr(o_out), D, _stream(stream)))
 
 
-def tm_debug_schedule(B, Hq, Hkv, N, causal, S, W, L, num_ctas=148, split=False) -> np.ndarray:
+def tm_debug_schedule(B, Hq, Hkv, N, causal, S, W, L, num_ctas=148, split=False,
+                      mix_pairs=False) -> np.ndarray:
     """Persistent work split as an int32 [n, 7] array:
     (cta, item, q-block, head0, Q tiles, first tile, end tile)."""
+    split = int(bool(split)) | (2 if mix_pairs else 0)
     cnt = ctypes.c_longlong(0)
     _check("tm_debug_schedule", lib().tm_debug_schedule(B, Hq, Hkv, N, int(causal), S, W, L,
                                                         num_ctas, int(split), None, 0,

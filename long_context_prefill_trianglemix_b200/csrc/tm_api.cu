@@ -3,6 +3,7 @@
 // All device work is delegated to tm_attn.cu.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -87,8 +88,11 @@ int scratch_address(void** out) {
 
 int run(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv, int N, int D,
         float scale, const trimix::Pattern& pat, void* ws, long long ws_bytes, void* stream,
-        const int* bs_off = nullptr, const int* bs_idx = nullptr, long long bs_nnz = 0) {
+        const int* bs_off = nullptr, const int* bs_idx = nullptr, long long bs_nnz = 0,
+        const int* hS = nullptr, const int* hW = nullptr) {
   trimix::LaunchArgs a;
+  a.hS = hS;
+  a.hW = hW;
   a.bs_off = bs_off;
   a.bs_idx = bs_idx;
   a.bs_nnz = bs_nnz;
@@ -155,6 +159,25 @@ TM_API int tm_trianglemix_attn_fwd(const void* q, const void* k, const void* v, 
                                    int layer, int tri_start, void* stream) {
   return tm_trianglemix_attn_fwd_ws(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L, layer,
                                     tri_start, nullptr, 0, stream);
+}
+
+TM_API int tm_triangle_attn_fwd_heads(const void* q, const void* k, const void* v, void* o, int B,
+                                      int Hq, int Hkv, int N, int D, float scale,
+                                      const int* S_heads, const int* W_heads, int L,
+                                      void* workspace, long long workspace_bytes, void* stream) {
+  if (int rc = validate_common(q, k, v, o, B, Hq, Hkv, N, D, scale)) return rc;
+  if (!S_heads || !W_heads || L < 0) return TM_ERR_INVALID_ARG;
+  if (Hq > 128) return TM_ERR_UNSUPPORTED;
+  int S_max = 0, W_max = 1;
+  for (int h = 0; h < Hq; ++h) {
+    if (S_heads[h] < 0 || W_heads[h] < 1) return TM_ERR_INVALID_ARG;
+    S_max = std::max(S_max, S_heads[h]);
+    W_max = std::max(W_max, W_heads[h]);
+  }
+  if (int rc = validate_workspace(q, k, v, o, B, Hq, Hkv, N, D, workspace, workspace_bytes))
+    return rc;
+  return run(q, k, v, o, B, Hq, Hkv, N, D, scale, trimix::make_pattern(N, 0, S_max, W_max, L),
+             workspace, workspace_bytes, stream, nullptr, nullptr, 0, S_heads, W_heads);
 }
 
 TM_API int tm_block_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o, int B,

@@ -69,6 +69,7 @@ static_assert(2 * 128 * kSoftmaxRegs + 128 * kSideRegs == kThreads * kLaunchRegs
 constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
 constexpr int kMaxCtas = 192;
+constexpr int kMaxBandHeads = 128;  // q heads of a per-head band launch
 constexpr uint32_t kTmemCols = 512;
 // Keep a stale running max until the true max exceeds it by 2^8: p stays <= 256
 // in fp32/bf16, and the O rescale (a TMEM round trip) becomes rare.
@@ -154,7 +155,9 @@ struct AttnParams {
   // all npairs values along its stride and every CTA gets its share of the
   // cheap single-tile items (0 for even group sizes). The rotation permutes
   // the pairs inside each (kv head, q-block) group, whose items stay adjacent.
-  int pair_rot;
+  // kv_rot rotates the kv head the same way (per-head band launches, whose kv
+  // heads differ in cost); it permutes whole groups, which stay adjacent too.
+  int pair_rot, kv_rot;
   // Split pieces (nsplit > 1): each writes its unnormalised partial (O, running
   // max m, sum l) of every 32-row warp slice to ws_rec and counts itself in
   // ws_cnt (one counter per cut item, Q tile and warp, zero at launch); the
@@ -168,6 +171,15 @@ struct AttnParams {
   const int* bs_off;
   const int* bs_idx;
   int bs_nnz;
+  // Per-head bands (ph != 0): q head h keeps the sinks [0, hS[h]) and a window
+  // of hW[h] positions (L and the rest of pat shared; pat.S, pat.W hold the
+  // maxima). The heads of each kv group are paired in the order hperm (sorted
+  // by band on the host, so the two heads of a pair have similar bands); an
+  // item visits the union of its two heads' tile lists, which is the closed
+  // form at (max S, max W) since both kept sets are [0, S) U [i - W + 1, i].
+  int ph;
+  int hS[kMaxBandHeads], hW[kMaxBandHeads];
+  unsigned char hperm[kMaxBandHeads];
 };
 
 __host__ __device__ __forceinline__ int big_count(const AttnParams& p, int c, int g) {
@@ -200,15 +212,42 @@ __host__ __device__ __forceinline__ int work_item(const AttnParams& p, int c, in
   return k < nb ? c + k * g : p.n_big + static_cast<int>(normal_index(p, c, g, k - nb));
 }
 
-// One unit of work: Q tiles h0 (and h0 + 1 if v1) of q-block qb, kv head g of
-// batch b, over tiles [t0, min(t1, count)) of the q-block's tile list. split
-// >= 0 marks a piece of a heavy item (hunit: its index among the heavy items).
+// One unit of work: Q tiles of q heads h0 (and h1 if v1) of q-block qb, kv
+// head g of batch b, over tiles [t0, min(t1, count)) of the q-block's tile
+// list. split >= 0 marks a piece of a heavy item (hunit: its index among the
+// heavy items).
 struct Item {
-  int b, g, qb, h0, v1;
+  int b, g, qb, h0, h1, v1;
   int t0, t1, split, hunit;
 };
 
 constexpr int kAllTiles = 0x7fffffff;
+
+// The q heads of pair pr of kv head g (h1 = h0 when the group ends in a single head).
+__host__ __device__ __forceinline__ void pair_heads(const AttnParams& p, int g, int pr, Item& it) {
+  const int hp = g * p.G + 2 * pr;
+  it.v1 = (2 * pr + 1 < p.G) ? 1 : 0;
+  it.h0 = p.ph ? p.hperm[hp] : hp;
+  it.h1 = it.v1 ? (p.ph ? p.hperm[hp + 1] : hp + 1) : it.h0;
+}
+
+// Pattern of one q head, and of an item (the union of its heads' patterns).
+__host__ __device__ __forceinline__ Pattern head_pattern(const AttnParams& p, int h) {
+  Pattern q = p.pat;
+  if (p.ph) {
+    q.S = p.hS[h];
+    q.W = p.hW[h];
+  }
+  return q;
+}
+__host__ __device__ __forceinline__ Pattern item_pattern(const AttnParams& p, const Item& it) {
+  Pattern q = p.pat;
+  if (p.ph) {
+    q.S = imax(p.hS[it.h0], p.hS[it.h1]);
+    q.W = imax(p.hW[it.h0], p.hW[it.h1]);
+  }
+  return q;
+}
 
 __host__ __device__ __forceinline__ Item decode_item(const AttnParams& p, int item) {
   Item it;
@@ -222,10 +261,9 @@ __host__ __device__ __forceinline__ Item decode_item(const AttnParams& p, int it
   const int pr = (u % p.npairs + static_cast<int>(static_cast<long long>(qi) * p.pair_rot % p.npairs)) %
                  p.npairs;
   const int gb = u / p.npairs;
-  it.g = gb % p.Hkv;
+  it.g = (gb % p.Hkv + static_cast<int>(static_cast<long long>(qi) * p.kv_rot % p.Hkv)) % p.Hkv;
   it.b = gb / p.Hkv;
-  it.h0 = it.g * p.G + 2 * pr;
-  it.v1 = (2 * pr + 1 < p.G) ? 1 : 0;
+  pair_heads(p, it.g, pr, it);
   it.t0 = 0;
   it.t1 = kAllTiles;
   it.split = -1;
@@ -245,7 +283,7 @@ __host__ __device__ __forceinline__ Item decode_piece(const AttnParams& p, int b
   const int u = rem - s * p.units;
   Item it = decode_item(p, qi * p.units + u);
   if (p.nsplit > 1) {
-    const int T = block_tiles(p.pat, it.qb, BM, BN).count();
+    const int T = block_tiles(item_pattern(p, it), it.qb, BM, BN).count();
     it.t0 = static_cast<int>(static_cast<long long>(T) * s / p.nsplit);
     it.t1 = static_cast<int>(static_cast<long long>(T) * (s + 1) / p.nsplit);
     it.split = s;
@@ -283,7 +321,7 @@ __device__ __forceinline__ TileSrc tile_src(const AttnParams& p, const Item& it)
     s.n = o1 - o0;
     s.bt.n_a = s.bt.b_lo = s.bt.n_b = 0;
   } else {
-    s.bt = block_tiles(p.pat, it.qb, BM, BN);
+    s.bt = block_tiles(item_pattern(p, it), it.qb, BM, BN);
   }
   return s;
 }
@@ -299,6 +337,7 @@ struct WorkCursor {
   int pr, kvh, b, qi;               // digits of the next normal item
   int d_pr, d_kvh, d_b, d_qi;       // digits of the current stride
   int rot, d_rot;                   // qi * pair_rot and d_qi * pair_rot, mod npairs
+  int krot, d_krot;                 // qi * kv_rot and d_qi * kv_rot, mod Hkv
   __host__ __device__ __forceinline__ void set_item(const AttnParams& p, long long item) {
     qi = static_cast<int>(item / p.units);
     const int u = static_cast<int>(item - static_cast<long long>(qi) * p.units);
@@ -307,6 +346,7 @@ struct WorkCursor {
     kvh = gb % p.Hkv;
     b = gb / p.Hkv;
     rot = static_cast<int>(static_cast<long long>(qi) * p.pair_rot % p.npairs);
+    krot = static_cast<int>(static_cast<long long>(qi) * p.kv_rot % p.Hkv);
   }
   __host__ __device__ __forceinline__ void set_stride(const AttnParams& p, int stride) {
     d_qi = stride / p.units;
@@ -316,6 +356,7 @@ struct WorkCursor {
     d_kvh = gb % p.Hkv;
     d_b = gb / p.Hkv;
     d_rot = static_cast<int>(static_cast<long long>(d_qi) * p.pair_rot % p.npairs);
+    d_krot = static_cast<int>(static_cast<long long>(d_qi) * p.kv_rot % p.Hkv);
   }
   __host__ __device__ __forceinline__ void enter_phase(const AttnParams& p) {
     set_item(p, p.n_hunits + normal_index(p, c, g, j));
@@ -346,12 +387,13 @@ struct WorkCursor {
       it.split = -1;
       it.hunit = -1;
       it.qb = p.nqb - 1 - qi;
-      it.g = kvh;
+      int ke = kvh + krot;
+      if (ke >= p.Hkv) ke -= p.Hkv;
+      it.g = ke;
       it.b = b;
       int pe = pr + rot;
       if (pe >= p.npairs) pe -= p.npairs;
-      it.h0 = kvh * p.G + 2 * pe;
-      it.v1 = (2 * pe + 1 < p.G) ? 1 : 0;
+      pair_heads(p, ke, pe, it);
       ++j;
       if (j == phase_end) {
         enter_phase(p);
@@ -369,6 +411,9 @@ struct WorkCursor {
         rot += d_rot + (carry ? p.pair_rot : 0);  // < 3 npairs
         if (rot >= p.npairs) rot -= p.npairs;
         if (rot >= p.npairs) rot -= p.npairs;
+        krot += d_krot + (carry ? p.kv_rot : 0);  // < 3 Hkv
+        if (krot >= p.Hkv) krot -= p.Hkv;
+        if (krot >= p.Hkv) krot -= p.Hkv;
       }
     }
     ++k;
@@ -479,7 +524,7 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, Bars<Cfg<D>::
       tma_load_4d(q0 + pn * Cfg<D>::kPanelBytes, tq, &bars->q_full, pn * 64, it.h0, it.qb * BM, it.b);
       if (it.v1)
         tma_load_4d(q0 + Cfg<D>::kTileBytes + pn * Cfg<D>::kPanelBytes, tq, &bars->q_full, pn * 64,
-                    it.h0 + 1, it.qb * BM, it.b);
+                    it.h1, it.qb * BM, it.b);
     }
     ++it_cnt;
     for (int t = it.t0; ok && t < t_end; ++t) {
@@ -682,7 +727,6 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
   const uint32_t tS = tmem_base + lane_addr + (wg ? Cfg<D>::kTmemS1 : Cfg<D>::kTmemS0);
   const uint32_t tO = tmem_base + lane_addr + (wg ? Cfg<D>::kTmemO1 : Cfg<D>::kTmemO0);
   const float sl2 = p.sl2;
-  const Pattern& pat = p.pat;
   uint32_t s_cnt = 0, o_cnt = 0;
   WorkCursor cur;
   cur.init(p, blockIdx.x, gridDim.x);
@@ -691,6 +735,8 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
     if (wg == 1 && !it.v1) continue;
     const TileSrc bt = tile_src(p, it);
     const int T = imin(bt.count(), it.t1) - it.t0;
+    const int head = wg ? it.h1 : it.h0;
+    const Pattern pat = head_pattern(p, head);  // this Q tile's own mask
     const int i = it.qb * BM + r;  // query row of this thread
     // kept keys of row i: [0, sink_hi) U [band_lo, hi)
     const int hi = imin(i, pat.N - 1) + 1;
@@ -832,8 +878,8 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
       }
       fence_proxy_async_smem();  // make the generic-proxy writes visible to the TMA engine
       __syncwarp();
-      if (lane == 0 && it.qb * BM + wq * 32 < pat.N) {  // a slot wholly past N stores nothing
-        tma_store_4d(to, slot, 64 * h, it.h0 + wg, it.qb * BM + wq * 32, it.b);
+      if (lane == 0 && it.qb * BM + wq * 32 < p.N) {  // a slot wholly past N stores nothing
+        tma_store_4d(to, slot, 64 * h, head, it.qb * BM + wq * 32, it.b);
         bulk_commit_group();
       }
     }
@@ -1100,7 +1146,7 @@ int encode_bnhd(CUtensorMap* m, const void* base, int B, int N, int H, int D, in
 // Fills the geometry and the persistent work split of *p; returns the grid
 // size. split: heavy items may be cut into pieces (the caller has workspace).
 int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ctas, bool split,
-                   AttnParams* p, bool sparse = false) {
+                   AttnParams* p, bool sparse = false, bool mix_pairs = false) {
   p->B = B; p->Hq = Hq; p->Hkv = Hkv; p->N = N;
   p->G = Hq / Hkv;
   p->npairs = (p->G + 1) / 2;
@@ -1110,9 +1156,11 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
   p->ws_rec = nullptr;
   p->ws_cnt = nullptr;
   p->pair_rot = 0;
+  p->kv_rot = 0;
   p->bs_off = nullptr;
   p->bs_idx = nullptr;
   p->bs_nnz = 0;
+  p->ph = 0;
   // Persistent grid. Item cost = (visited tiles + fixed per-item overhead,
   // about the pipeline fill/drain and epilogue) x Q tiles of the item; it is
   // used to find the heavy q-blocks, how finely to cut them, and how many
@@ -1158,18 +1206,22 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
   p->n_sqb = n_sqb;
   p->n_sbig = n_sqb * p->units * ns;
   p->n_big = p->n_sbig + (n_hqb - n_sqb) * p->units;
-  if (p->G % 2 == 1 && p->npairs > 1) {
-    // per stride of grid items the pair digit advances by d_pr (plus carries)
-    // and the q-block slot by d_qi; take the first rotation that makes the
-    // advance coprime with npairs
-    const int d_qi = grid / p->units;
-    const int d_pr = (grid % p->units) % p->npairs;
-    for (int r = 0; r < p->npairs; ++r) {
-      int a = (d_pr + d_qi * r) % p->npairs, b = p->npairs;
+  // per stride of grid items a digit of radix n advances by d (plus carries)
+  // and the q-block slot by d_qi; the first rotation r that makes d + d_qi * r
+  // coprime with n lets that digit run through all its values
+  auto coprime_rotation = [](int d, int d_qi, int n) {
+    for (int r = 0; r < n; ++r) {
+      int a = (d + d_qi * r) % n, b = n;
       while (b) { const int t = a % b; a = b; b = t; }
-      if (a == 1) { p->pair_rot = r; break; }
+      if (a == 1) return r;
     }
-  }
+    return 0;
+  };
+  const int d_qi = grid / p->units;
+  if ((p->G % 2 == 1 || mix_pairs) && p->npairs > 1)
+    p->pair_rot = coprime_rotation((grid % p->units) % p->npairs, d_qi, p->npairs);
+  if (mix_pairs && p->Hkv > 1)
+    p->kv_rot = coprime_rotation((grid % p->units) / p->npairs % p->Hkv, d_qi, p->Hkv);
   p->n_a = 0;
   p->n_skip = 0;
   const long long n_norm = n_items - p->n_hunits;
@@ -1233,9 +1285,27 @@ int launch_attention_d(const LaunchArgs& a, DeviceInfo* di) {
 
   AttnParams p;
   const bool sparse = a.bs_off != nullptr;
-  const int grid =
-      build_schedule(a.B, a.Hq, a.Hkv, a.N, a.pat, di->sms, a.ws != nullptr, &p, sparse);
+  // per-head bands: pairs differ in cost, so every CTA cycles through the pairs
+  const int grid = build_schedule(a.B, a.Hq, a.Hkv, a.N, a.pat, di->sms, a.ws != nullptr, &p,
+                                  sparse, a.hS != nullptr);
   p.sl2 = a.scale * 1.4426950408889634f;
+  if (a.hS) {  // per-head bands; a.pat already holds the maxima
+    if (a.Hq > kMaxBandHeads) return TM_ERR_UNSUPPORTED;
+    p.ph = 1;
+    for (int h = 0; h < a.Hq; ++h) {
+      p.hS[h] = std::min(std::max(a.hS[h], 0), a.N);
+      p.hW[h] = std::min(std::max(a.hW[h], 1), a.N);
+    }
+    const int G = a.Hq / a.Hkv;
+    std::vector<int> order(G);
+    for (int g = 0; g < a.Hkv; ++g) {  // pair the heads of a group in band order
+      for (int x = 0; x < G; ++x) order[x] = g * G + x;
+      std::stable_sort(order.begin(), order.end(), [&](int u, int v) {
+        return p.hW[u] != p.hW[v] ? p.hW[u] < p.hW[v] : p.hS[u] < p.hS[v];
+      });
+      for (int x = 0; x < G; ++x) p.hperm[g * G + x] = static_cast<unsigned char>(order[x]);
+    }
+  }
   if (sparse) {
     p.bs_off = a.bs_off;
     p.bs_idx = a.bs_idx;
@@ -1368,7 +1438,8 @@ int workspace_bytes(int B, int Hq, int Hkv, int N, int D, const Pattern& pat, in
 int debug_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ctas, int split,
                    int* out, long long cap, long long* count) {
   AttnParams p;
-  const int grid = build_schedule(B, Hq, Hkv, N, pat, max_ctas, split != 0, &p);
+  const int grid =
+      build_schedule(B, Hq, Hkv, N, pat, max_ctas, (split & 1) != 0, &p, false, (split & 2) != 0);
   long long n = 0;
   for (int c = 0; c < grid; ++c) {
     WorkCursor cur;
@@ -1379,7 +1450,8 @@ int debug_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
       const int item = work_item(p, c, grid, k);
       const Item ref = item < p.n_big ? decode_piece(p, item)
                                       : decode_item(p, item - p.n_big + p.n_hunits);
-      if (it.qb != ref.qb || it.b != ref.b || it.g != ref.g || it.h0 != ref.h0 || it.v1 != ref.v1 ||
+      if (it.qb != ref.qb || it.b != ref.b || it.g != ref.g || it.h0 != ref.h0 || it.h1 != ref.h1 ||
+          it.v1 != ref.v1 ||
           it.t0 != ref.t0 || it.t1 != ref.t1 || it.split != ref.split || it.hunit != ref.hunit)
         return TM_ERR_INVALID_ARG;  // the cursor and the direct decode disagree
       if (n >= cap) continue;

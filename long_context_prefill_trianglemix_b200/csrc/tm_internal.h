@@ -24,6 +24,8 @@ struct LaunchArgs {
   const int* bs_off;  // block-sparse index (device CSR), or nullptr: pat's tile list
   const int* bs_idx;
   long long bs_nnz;
+  const int* hS;      // per-head sinks and windows (host, Hq each), or nullptr
+  const int* hW;
   void* stream;
 };
 

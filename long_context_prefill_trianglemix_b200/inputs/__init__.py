@@ -337,3 +337,15 @@ def full_causal_index(B: int, Hkv: int, N: int, BM: int = 128):
     offsets = np.zeros(len(per) + 1, np.int32)
     offsets[1:] = np.cumsum([len(x) for x in per])
     return offsets, np.fromiter((c for x in per for c in x), np.int32, count=int(offsets[-1]))
+
+
+def head_bands(Hq: int, seed: int, w_min: int = 512, w_max: int = 4096, sinks=(0, 64)):
+    """Seeded per-head (S_h, W_h): windows log-uniform in [w_min, w_max], sinks
+    drawn from ``sinks`` (a calibrated policy stands in for nothing here; this
+    only spreads the bands the way per-head calibration would)."""
+    S = np.array([sinks[int(_uniform(seed, 5000, h) * len(sinks)) % len(sinks)]
+                  for h in range(Hq)], np.int32)
+    lo, hi = np.log(w_min), np.log(w_max)
+    W = np.array([int(round(np.exp(lo + (hi - lo) * _uniform(seed, 5001, h)))) for h in range(Hq)],
+                 np.int32)
+    return S, W

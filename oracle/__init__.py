@@ -48,6 +48,9 @@ def _load():
         lib.oracle_block_sparse_attention.argtypes = [
             vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_dbl, c_int, c_int, vp, vp, c_ll, vp,
             c_ll, vp, c_int]
+        lib.oracle_attention_heads.restype = c_int
+        lib.oracle_attention_heads.argtypes = [vp, vp, vp, c_int, c_int, c_int, c_int, c_int,
+                                               c_dbl, vp, vp, c_int, vp, c_ll, vp, c_int]
         lib.oracle_flashprefill_scores.restype = c_int
         lib.oracle_flashprefill_scores.argtypes = [vp, vp, c_int, c_int, c_int, c_int, c_int,
                                                    c_dbl, c_int, c_int, vp, c_int]
@@ -189,3 +192,26 @@ def flashprefill_select(scores, alpha):
     off = np.zeros(len(lists) + 1, np.int32)
     off[1:] = np.cumsum([len(x) for x in lists])
     return off, (np.concatenate(lists) if lists else np.zeros(0, np.int32))
+
+
+def attention_heads(q, k, v, B, Hq, Hkv, N, D, scale, S_heads, W_heads, L, rows=None,
+                    nthreads=None):
+    """fp64 triangle attention with per-head sinks S_heads[h] and windows W_heads[h]."""
+    lib = _load()
+    for a in (q, k, v):
+        assert a.dtype == np.uint16 and a.flags.c_contiguous
+    Sh = np.ascontiguousarray(S_heads, dtype=np.int32)
+    Wh = np.ascontiguousarray(W_heads, dtype=np.int32)
+    assert Sh.size == Hq and Wh.size == Hq
+    if rows is None:
+        nrows, rows_ptr = N, None
+    else:
+        rows_arr = np.ascontiguousarray(rows, dtype=np.int64)
+        nrows, rows_ptr = len(rows_arr), rows_arr.ctypes.data
+    out = np.zeros((B, nrows, Hq, D), np.float64)
+    rc = lib.oracle_attention_heads(q.ctypes.data, k.ctypes.data, v.ctypes.data, B, Hq, Hkv, N, D,
+                                    float(scale), Sh.ctypes.data, Wh.ctypes.data, L, rows_ptr,
+                                    nrows, out.ctypes.data, nthreads or hardware_threads())
+    if rc != 0:
+        raise ValueError("oracle_attention_heads: bad argument")
+    return out

@@ -34,7 +34,9 @@
 //     q = 0 gives the mean of v over the kept keys; rows match the library
 //     routine under a block mask built independently; empty lists give 0;
 //   * discovery scores: q = 0 gives 1 / (I + 1); one probe on one head gives
-//     a plain softmax (a worked example with closed-form values).
+//     a plain softmax (a worked example with closed-form values);
+//   * per-head bands: every head equals the single-pattern oracle run with
+//     that head's sinks and window; equal bands give the shared-band result.
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
@@ -351,6 +353,69 @@ int oracle_flashprefill_scores(const uint16_t* q, const uint16_t* k, int B, int 
         }
       double* out = scores + (bg * nb + I) * nb;
       for (long long J = 0; J < nb; ++J) out[J] = J <= I ? mean[size_t(J)] / double(G * P) : 0.0;
+    }
+  });
+  return 0;
+}
+
+// Triangle attention with a band per q head (the bf16 reading of the
+// TriAttention page's per-head regions bounded by diagonal distances): head h
+// keeps j <= i and (j < S_h or i - j < W_h or i >= N - L). For every (b, i, h)
+// the mask row is built explicitly from head h's pattern and the attention is
+// the same fp64 computation as oracle_attention. S_h, W_h: Hq ints each.
+// Returns 0, or -1 on a bad argument.
+int oracle_attention_heads(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq,
+                           int Hkv, int N, int D, double scale, const int* S_h, const int* W_h,
+                           int L, const long long* rows, long long nrows, double* out,
+                           int nthreads) {
+  if (!q || !k || !v || !out || !S_h || !W_h || B < 1 || Hq < 1 || Hkv < 1 || D < 1 ||
+      Hq % Hkv != 0)
+    return -1;
+  std::vector<Pattern> pats(static_cast<size_t>(Hq));
+  for (int h = 0; h < Hq; ++h)
+    if (!make_pattern(N, 0, S_h[h], W_h[h], L, &pats[size_t(h)])) return -1;
+  if (!rows) nrows = N;
+  if (nrows < 0) return -1;
+  for (long long r = 0; rows && r < nrows; ++r)
+    if (rows[r] < 0 || rows[r] >= N) return -1;
+  const int G = Hq / Hkv;
+  parallel_for((long long)B * nrows, nthreads, [&](long long ub, long long ue) {
+    std::vector<unsigned char> m;
+    std::vector<long long> idx;
+    std::vector<double> s, qrow(static_cast<size_t>(D)), o(static_cast<size_t>(D));
+    for (long long u = ub; u < ue; ++u) {
+      const long long b = u / nrows, r = u % nrows;
+      const long long i = rows ? rows[r] : r;
+      for (int hq = 0; hq < Hq; ++hq) {
+        const int g = hq / G;
+        mask_row(pats[size_t(hq)], i, m);  // explicit mask row of this head
+        idx.clear();
+        for (long long j = 0; j < N; ++j)
+          if (m[size_t(j)]) idx.push_back(j);
+        s.resize(idx.size());
+        const uint16_t* qp = q + ((b * N + i) * Hq + hq) * (long long)D;
+        for (int d = 0; d < D; ++d) qrow[size_t(d)] = bf16_to_double(qp[d]);
+        double mx = -std::numeric_limits<double>::infinity();
+        for (size_t t = 0; t < idx.size(); ++t) {
+          const uint16_t* kp = k + ((b * N + idx[t]) * Hkv + g) * (long long)D;
+          double acc = 0.0;
+          for (int d = 0; d < D; ++d) acc += qrow[size_t(d)] * bf16_to_double(kp[d]);
+          s[t] = scale * acc;
+          mx = std::max(mx, s[t]);
+        }
+        double l = 0.0;
+        for (size_t t = 0; t < idx.size(); ++t) {
+          s[t] = std::exp(s[t] - mx);
+          l += s[t];
+        }
+        std::fill(o.begin(), o.end(), 0.0);
+        for (size_t t = 0; t < idx.size(); ++t) {
+          const uint16_t* vp = v + ((b * N + idx[t]) * Hkv + g) * (long long)D;
+          for (int d = 0; d < D; ++d) o[size_t(d)] += s[t] * bf16_to_double(vp[d]);
+        }
+        double* op = out + ((b * nrows + r) * Hq + hq) * (long long)D;
+        for (int d = 0; d < D; ++d) op[d] = o[size_t(d)] / l;
+      }
     }
   });
   return 0;

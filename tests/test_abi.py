@@ -178,3 +178,25 @@ def test_block_sparse_validation():
     # the triangle branch ignores the index but still checks the pattern
     assert L.tm_trianglemix_sparse_attn_fwd(*args, 4, 0, 2, 3, 1, None, None, 0,
                                             None) == tm.TM_ERR_INVALID_ARG
+
+
+def test_per_head_band_validation():
+    L = tm.lib()
+    args = (FAKE, FAKE, FAKE, FAKE + 0x100000, 1, 4, 4, 64, 64, 0.1)
+    good = (ctypes.c_int * 4)(1, 2, 3, 4)
+    bad_w = (ctypes.c_int * 4)(1, 0, 3, 4)
+    bad_s = (ctypes.c_int * 4)(1, -2, 3, 4)
+    assert L.tm_triangle_attn_fwd_heads(*args, None, good, 2, None, 0, None) == tm.TM_ERR_INVALID_ARG
+    assert L.tm_triangle_attn_fwd_heads(*args, good, bad_w, 2, None, 0, None) == tm.TM_ERR_INVALID_ARG
+    assert L.tm_triangle_attn_fwd_heads(*args, bad_s, good, 2, None, 0, None) == tm.TM_ERR_INVALID_ARG
+    assert L.tm_triangle_attn_fwd_heads(*args, good, good, -1, None, 0, None) == tm.TM_ERR_INVALID_ARG
+
+
+def test_seeded_head_bands():
+    from long_context_prefill_trianglemix_b200 import inputs as I
+    S, W = I.head_bands(32, 0)
+    assert S.shape == (32,) and W.shape == (32,)
+    assert set(S.tolist()) <= {0, 64} and (W >= 512).all() and (W <= 4096).all()
+    assert len(set(W.tolist())) > 20
+    S2, W2 = I.head_bands(32, 0)
+    assert np.array_equal(S, S2) and np.array_equal(W, W2)

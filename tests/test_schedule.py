@@ -170,3 +170,24 @@ def test_items_of_one_kv_head_and_q_block_are_adjacent(B, Hq, Hkv, N, causal, W,
     for key, items in groups.items():
         assert len(items) == npairs
         assert max(items) - min(items) == npairs - 1, (key, sorted(items))
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,causal,S,W,L", CASES[:12] + SPLIT_CASES[:4])
+def test_pair_and_kv_rotation_keep_exact_coverage(B, Hq, Hkv, N, causal, S, W, L):
+    # per-head band launches rotate the pair and kv-head digits per q-block; the
+    # host export cross-checks the device cursor against the direct decode, and
+    # every (q-block, head) must still be covered exactly once, with the items of
+    # one kv head and q-block adjacent
+    for split in (False, True):
+        rec = tm.tm_debug_schedule(B, Hq, Hkv, N, causal, S, W, L, 148, split=split, mix_pairs=True)
+        tiles = tm.tm_tile_list(N, causal, S, W, L)
+        per_qb = np.bincount(tiles[:, 0], minlength=(N + 127) // 128)
+        seen = {}
+        for c, item, qb, h0, nv, t0, t1 in rec:
+            for h in range(h0, h0 + nv):
+                seen.setdefault((qb, h), []).append((t0, t1))
+        assert len(seen) == ((N + 127) // 128) * B * Hq
+        for (qb, h), ranges in seen.items():
+            ranges.sort()
+            assert ranges[0][0] == 0 and ranges[-1][1] == per_qb[qb]
+            assert all(a1 == b0 for (_, a1), (b0, _) in zip(ranges, ranges[1:]))
