@@ -40,7 +40,7 @@ BM = BN = 128
 # triangle launch of the default workload (llama3-8b-128k, W=2048) from one ncu
 # capture of this bench command, keyed by the hash of the kernel sources it was
 # taken on; reported only while the sources still match (else null).
-TRAFFIC = {"1807816c69e24010": 2.45e9 + 1.045e9}
+TRAFFIC = {"ed93a8ae342f5c84": 2.215e9 + 1.041e9}
 
 
 def kernel_source_hash() -> str:
