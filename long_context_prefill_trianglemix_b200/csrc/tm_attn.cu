@@ -127,7 +127,12 @@ struct Bars {
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
+  // The producer's item descriptor for the MMA issuer: visited tiles (0 ends
+  // the CTA's work) and whether a second Q tile is present. Written before the
+  // producer's arrival on q_full, read after the issuer's wait on it.
+  int item_T, item_v1;
 };
+static_assert(sizeof(Bars<8>) <= 256 && sizeof(Bars<4>) <= 256, "barrier block is 256 bytes");
 
 struct AttnParams {
   int B, Hq, Hkv, N, G, npairs, nqb, units;
@@ -518,6 +523,8 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, Bars<Cfg<D>::
     const int t_end = imin(bt.count(), it.t1);
     if (t_end <= it.t0) continue;  // an empty block-sparse list: nothing to load
     if (!(ok = wait_bar(&bars->q_empty, (it_cnt & 1u) ^ 1u, abort_flag, kSiteQEmpty))) break;
+    bars->item_T = t_end - it.t0;
+    bars->item_v1 = it.v1;
     mbar_arrive_expect_tx(&bars->q_full, (1 + it.v1) * Cfg<D>::kTileBytes);
 #pragma unroll
     for (int pn = 0; pn < Cfg<D>::kPanels; ++pn) {
@@ -544,6 +551,13 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, Bars<Cfg<D>::
       }
     }
   }
+  if (ok) {  // no more items: a descriptor of zero tiles, once Q is released
+    if ((ok = wait_bar(&bars->q_empty, (it_cnt & 1u) ^ 1u, abort_flag, kSiteQEmpty))) {
+      bars->item_T = 0;
+      bars->item_v1 = 0;
+      mbar_arrive(&bars->q_full);
+    }
+  }
   if (!ok) {  // let copies already in flight land before the CTA goes away
     const uint32_t first = kv_cnt > (uint32_t)NST ? kv_cnt - NST : 0;
     for (uint32_t idx = first; idx < kv_cnt; ++idx)
@@ -553,7 +567,14 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, Bars<Cfg<D>::
 }
 
 // The tcgen05 issuer: one thread issues every MMA of both Q tiles in the order
-// O0+=P0.V_t, S0=Q0.K_{t+1}, O1+=P1.V_t, S1=Q1.K_{t+1}. Descriptors are kept as
+// O0+=P0.V_t, S0=Q0.K_{t+1}, O1+=P1.V_t, S1=Q1.K_{t+1}, and keeps that order
+// across item boundaries: after the last O0+=P0.V of an item it issues the
+// next item's first S0 (then, after O1+=P1.V, its S1), so one softmax
+// warpgroup starts the next item while the tensor core finishes the other's
+// products. (The next Q is loaded once the current item's last S is done;
+// K/V arrive in the ring in exactly this order; the producer publishes each
+// item's tile count with its Q, and a zero count after the last item.)
+// Descriptors are kept as
 // precomputed low words plus per-k-step constant adds: the issuing warp shares
 // its SM sub-partition with two softmax warps, so every instruction it saves
 // per MMA shortens the time the tensor pipe waits for the next one.
@@ -574,27 +595,37 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStag
 #define TM_WAIT(bar, par, site)                                      \
   if (!(ok = wait_bar((bar), (par), abort_flag, (site)))) break; \
   tc_fence_after();
-  WorkCursor cur;
-  cur.init(p, blockIdx.x, gridDim.x);
-  while (ok && !cur.done()) {
-    const Item it = cur.next(p);
-    const int T = imin(tile_src(p, it).count(), it.t1) - it.t0;
-    if (T <= 0) continue;  // an empty block-sparse list
-    const bool v1 = it.v1 != 0;
-    TM_WAIT(&bars->q_full, it_cnt & 1u, kSiteQFull);
-    ++it_cnt;
-    uint32_t kst = kv_cnt % NST;
-    TM_WAIT(&bars->kv_full[kst], (kv_cnt / NST) & 1u, kSiteKvFull);
-    issue_qk<D>(tS0, q0, k_lo0 + kst * kStageLo);
-    mma_commit(&bars->s_full[0]);
-    if (v1) {
-      issue_qk<D>(tS1, q1, k_lo0 + kst * kStageLo);
-      mma_commit(&bars->s_full[1]);
+  // Items come from the producer's descriptors (no work cursor here: the
+  // issuer's registers are few and its loop is on the critical path).
+  if (!(ok = wait_bar(&bars->q_full, it_cnt & 1u, abort_flag, kSiteQFull))) {
+    mma_commit(&bars->mma_done);
+    drain_wait(&bars->mma_done, 0);
+    return;
+  }
+  tc_fence_after();
+  ++it_cnt;
+  int T = bars->item_T;
+  bool v1 = bars->item_v1 != 0;
+  bool started = false;  // this item's first S products were issued by the previous item's tail
+  uint32_t kst = 0;
+  while (ok && T > 0) {
+    if (!started) {
+      kst = kv_cnt % NST;
+      TM_WAIT(&bars->kv_full[kst], (kv_cnt / NST) & 1u, kSiteKvFull);
+      issue_qk<D>(tS0, q0, k_lo0 + kst * kStageLo);
+      mma_commit(&bars->s_full[0]);
+      if (v1) {
+        issue_qk<D>(tS1, q1, k_lo0 + kst * kStageLo);
+        mma_commit(&bars->s_full[1]);
+      }
+      if (T == 1) mma_commit(&bars->q_empty);
+      mma_commit(&bars->kv_empty[kst]);
+      ++kv_cnt;
     }
-    if (T == 1) mma_commit(&bars->q_empty);
-    mma_commit(&bars->kv_empty[kst]);
-    ++kv_cnt;
-    for (int t = 0; t < T; ++t) {
+    int Tn = 0;
+    bool v1n = false;
+    // steady state: tiles 0 .. T-2 (the next S of each is this item's tile t+1)
+    for (int t = 0; t + 1 < T; ++t) {
       const uint32_t vst = kv_cnt % NST;
       TM_WAIT(&bars->kv_full[vst], (kv_cnt / NST) & 1u, kSiteKvFull);
       if (t == 0) {
@@ -606,14 +637,61 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStag
       TM_WAIT(&bars->p_full[1], pc0 & 1u, kSitePFull);
       ++pc0;
       issue_pv<D, 4, 8>(tO0, tS0, v_lo0 + vst * kStageLo, 1u);
-      if (t == T - 1) mma_commit(&bars->o_full[0]);
-      if (t + 1 < T) {
+      const uint32_t kidx = kv_cnt + 1;
+      kst = kidx % NST;
+      TM_WAIT(&bars->kv_full[kst], (kidx / NST) & 1u, kSiteKvFull);
+      issue_qk<D>(tS0, q0, k_lo0 + kst * kStageLo);
+      mma_commit(&bars->s_full[0]);
+      if (!v1 && t + 1 == T - 1) mma_commit(&bars->q_empty);
+      if (v1) {
+        if (t == 0) {
+          TM_WAIT(&bars->o_empty[1], (oe1 & 1u) ^ 1u, kSiteOEmpty);
+          ++oe1;
+        }
+        TM_WAIT(&bars->p_full[2], pc1 & 1u, kSitePFull);
+        issue_pv<D, 0, 4>(tO1, tS1, v_lo0 + vst * kStageLo, t > 0 ? 1u : 0u);
+        TM_WAIT(&bars->p_full[3], pc1 & 1u, kSitePFull);
+        ++pc1;
+        issue_pv<D, 4, 8>(tO1, tS1, v_lo0 + vst * kStageLo, 1u);
+      }
+      mma_commit(&bars->kv_empty[vst]);  // V_t free once both P.V products are done
+      ++kv_cnt;
+      if (v1) {
+        issue_qk<D>(tS1, q1, k_lo0 + kst * kStageLo);
+        mma_commit(&bars->s_full[1]);
+        if (t + 1 == T - 1) mma_commit(&bars->q_empty);
+      }
+      mma_commit(&bars->kv_empty[kst]);  // K_{t+1} free once both Q.K products are done
+      ++kv_cnt;
+    }
+    if (!ok) break;
+    // last tile: its products, with the next item's first S products in between
+    do {
+      const int t = T - 1;
+      const uint32_t vst = kv_cnt % NST;
+      TM_WAIT(&bars->kv_full[vst], (kv_cnt / NST) & 1u, kSiteKvFull);
+      if (t == 0) {
+        TM_WAIT(&bars->o_empty[0], (oe0 & 1u) ^ 1u, kSiteOEmpty);
+        ++oe0;
+      }
+      TM_WAIT(&bars->p_full[0], pc0 & 1u, kSitePFull);
+      issue_pv<D, 0, 4>(tO0, tS0, v_lo0 + vst * kStageLo, t > 0 ? 1u : 0u);
+      TM_WAIT(&bars->p_full[1], pc0 & 1u, kSitePFull);
+      ++pc0;
+      issue_pv<D, 4, 8>(tO0, tS0, v_lo0 + vst * kStageLo, 1u);
+      mma_commit(&bars->o_full[0]);
+      // the next item's descriptor (and Q), then its S0
+      TM_WAIT(&bars->q_full, it_cnt & 1u, kSiteQFull);
+      ++it_cnt;
+      Tn = bars->item_T;
+      v1n = bars->item_v1 != 0;
+      if (Tn > 0) {
         const uint32_t kidx = kv_cnt + 1;
         kst = kidx % NST;
         TM_WAIT(&bars->kv_full[kst], (kidx / NST) & 1u, kSiteKvFull);
         issue_qk<D>(tS0, q0, k_lo0 + kst * kStageLo);
         mma_commit(&bars->s_full[0]);
-        if (!v1 && t + 1 == T - 1) mma_commit(&bars->q_empty);
+        if (!v1n && Tn == 1) mma_commit(&bars->q_empty);
       }
       if (v1) {
         if (t == 0) {
@@ -625,20 +703,24 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStag
         TM_WAIT(&bars->p_full[3], pc1 & 1u, kSitePFull);
         ++pc1;
         issue_pv<D, 4, 8>(tO1, tS1, v_lo0 + vst * kStageLo, 1u);
-        if (t == T - 1) mma_commit(&bars->o_full[1]);
+        mma_commit(&bars->o_full[1]);
       }
-      mma_commit(&bars->kv_empty[vst]);  // V_t free once both P.V products are done
+      mma_commit(&bars->kv_empty[vst]);
       ++kv_cnt;
-      if (t + 1 < T) {
-        if (v1) {
+      if (Tn > 0) {
+        if (v1n) {
           issue_qk<D>(tS1, q1, k_lo0 + kst * kStageLo);
           mma_commit(&bars->s_full[1]);
-          if (t + 1 == T - 1) mma_commit(&bars->q_empty);
+          if (Tn == 1) mma_commit(&bars->q_empty);
         }
-        mma_commit(&bars->kv_empty[kst]);  // K_{t+1} free once both Q.K products are done
+        mma_commit(&bars->kv_empty[kst]);
         ++kv_cnt;
       }
-    }
+    } while (false);
+    if (!ok) break;
+    T = Tn;
+    v1 = v1n;
+    started = true;
   }
 #undef TM_WAIT
   // Every MMA issued above must finish before TMEM is released.
