@@ -517,11 +517,33 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, Bars<Cfg<D>::
   bool ok = true;
   WorkCursor cur;
   cur.init(p, blockIdx.x, gridDim.x);
+  // Per item: the first K/V tile goes into the ring before the wait for the Q
+  // buffer (its ring slot frees about a tile earlier than the previous item's
+  // last S releases Q, so it is in flight before Q), then Q, then the other
+  // tiles. The ring order the issuer consumes is unchanged. (An L2 prefetch of
+  // the next item's Q on top of this measured within noise and was dropped.)
+  auto load_kv = [&](const Item& it, const TileSrc& bt, int t) -> bool {
+    const int kb = bt.kb(t);
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      const uint32_t st = kv_cnt % NST;
+      if (!wait_bar(&bars->kv_empty[st], ((kv_cnt / NST) & 1u) ^ 1u, abort_flag, kSiteKvEmpty))
+        return false;
+      mbar_arrive_expect_tx(&bars->kv_full[st], Cfg<D>::kTileBytes);
+#pragma unroll
+      for (int pn = 0; pn < Cfg<D>::kPanels; ++pn)
+        tma_load_4d(ring + st * Cfg<D>::kTileBytes + pn * Cfg<D>::kPanelBytes, which ? tv : tk,
+                    &bars->kv_full[st], pn * 64, it.g, kb * BN, it.b);
+      ++kv_cnt;
+    }
+    return true;
+  };
   while (ok && !cur.done()) {
     const Item it = cur.next(p);
     const TileSrc bt = tile_src(p, it);
     const int t_end = imin(bt.count(), it.t1);
     if (t_end <= it.t0) continue;  // an empty block-sparse list: nothing to load
+    if (!(ok = load_kv(it, bt, it.t0))) break;
     if (!(ok = wait_bar(&bars->q_empty, (it_cnt & 1u) ^ 1u, abort_flag, kSiteQEmpty))) break;
     bars->item_T = t_end - it.t0;
     bars->item_v1 = it.v1;
@@ -534,22 +556,7 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, Bars<Cfg<D>::
                     it.h1, it.qb * BM, it.b);
     }
     ++it_cnt;
-    for (int t = it.t0; ok && t < t_end; ++t) {
-      const int kb = bt.kb(t);
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t st = kv_cnt % NST;
-        if (!(ok = wait_bar(&bars->kv_empty[st], ((kv_cnt / NST) & 1u) ^ 1u, abort_flag,
-                            kSiteKvEmpty)))
-          break;
-        mbar_arrive_expect_tx(&bars->kv_full[st], Cfg<D>::kTileBytes);
-#pragma unroll
-        for (int pn = 0; pn < Cfg<D>::kPanels; ++pn)
-          tma_load_4d(ring + st * Cfg<D>::kTileBytes + pn * Cfg<D>::kPanelBytes, which ? tv : tk,
-                      &bars->kv_full[st], pn * 64, it.g, kb * BN, it.b);
-        ++kv_cnt;
-      }
-    }
+    for (int t = it.t0 + 1; ok && t < t_end; ++t) ok = load_kv(it, bt, t);
   }
   if (ok) {  // no more items: a descriptor of zero tiles, once Q is released
     if ((ok = wait_bar(&bars->q_empty, (it_cnt & 1u) ^ 1u, abort_flag, kSiteQEmpty))) {
