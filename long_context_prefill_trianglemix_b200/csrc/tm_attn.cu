@@ -1264,12 +1264,20 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
   }
   const double target = static_cast<double>(total) / grid;
   // heavy q-blocks: from the top, while an item of the block costs more than a
-  // quarter of a CTA's share (at most 8 big items per CTA)
+  // quarter of a CTA's share, or more than twice the median q-block (a
+  // CTA that drew such an item in the strided rounds would carry its excess;
+  // dealt first, its holders join the rounds late instead); at most 8 big
+  // items per CTA
   const long long item_q = p->G >= 2 ? 2 : 1;
+  std::vector<long long> sorted_cost(qcost);
+  std::nth_element(sorted_cost.begin(), sorted_cost.begin() + p->nqb / 2, sorted_cost.end());
+  const long long median = sorted_cost[p->nqb / 2];
   // (block-sparse launches: costs are in device memory, every item is dealt
   // in the strided rounds, q-blocks from the last)
   int n_hqb = 0;
-  while (!sparse && n_hqb < p->nqb - 1 && 4.0 * qcost[p->nqb - 1 - n_hqb] * item_q > target &&
+  while (!sparse && n_hqb < p->nqb - 1 &&
+         (4.0 * qcost[p->nqb - 1 - n_hqb] * item_q > target ||
+          qcost[p->nqb - 1 - n_hqb] > 2 * median) &&
          static_cast<long long>(n_hqb + 1) * p->units <= 8LL * grid)
     ++n_hqb;
   p->n_hqb = n_hqb;

@@ -191,3 +191,16 @@ def test_pair_and_kv_rotation_keep_exact_coverage(B, Hq, Hkv, N, causal, S, W, L
             ranges.sort()
             assert ranges[0][0] == 0 and ranges[-1][1] == per_qb[qb]
             assert all(a1 == b0 for (_, a1), (b0, _) in zip(ranges, ranges[1:]))
+
+
+@pytest.mark.parametrize("W", [512, 2048, 4096, 8192, 16384, 32768])
+def test_wide_windows_keep_last_rows_as_big_items(W):
+    # The last-L q-blocks cost ~1024 tiles; with wide windows that is only a few
+    # percent of a CTA's share, but as a normal item it would land on a handful
+    # of CTAs; they count as big items once they cost twice the median q-block.
+    N, L = 131072, 256
+    per_qb = np.bincount(tm.tm_tile_list(N, False, 64, W, L)[:, 0], minlength=N // 128)
+    for split in (False, True):
+        rec = tm.tm_debug_schedule(1, 32, 8, N, False, 64, W, L, 148, split=split)
+        cost = cta_costs(rec, per_qb)
+        assert cost.max() <= 1.02 * cost.mean(), (W, split, cost.max() / cost.mean())
