@@ -292,3 +292,39 @@ def test_qwen_128k_two_layers_sampled():
         rows = sample_rows(wl.N, wl.L, 5 + layer, 32, 32 if causal else 96,
                            n_last=16 if causal else None)
         check_rows(o, host, wl, causal, rows, what=f"qwen 128K layer {layer}")
+
+
+def test_256k_context_sampled_rows_and_zero_query_every_row():
+    """The longest context in the pages' experiments (the FlashPrefill summary
+    reports 256K): N = 262144 with the Llama group shape on 8 q heads, the
+    split schedule on, sampled rows (all last-L rows) against the oracle and
+    the q = 0 closed form on every row."""
+    import dataclasses
+    import torch
+    wl = dataclasses.replace(I.WORKLOADS["llama3-8b-128k"], N=262144, Hq=8, Hkv=2)
+    q, k, v = I.make_qkv(wl)
+    dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
+    n = tm.tm_attn_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.N, wl.D, False, wl.S, wl.W, wl.L)
+    ws = torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
+    o = torch.empty_like(dq)
+    tm.tm_triangle_attn_fwd_ws(dq, dk, dv, o, wl.B, wl.Hq, wl.Hkv, wl.N, wl.D, wl.scale, wl.S,
+                               wl.W, wl.L, ws, n)
+    torch.cuda.synchronize()
+    assert tm.tm_get_device_status() == tm.TM_OK
+    rows = sample_rows(wl.N, wl.L, 13, 16, 48, n_last=64)
+    check_rows(o, (q, k, v), wl, False, rows, what="256K triangle")
+    zq = torch.zeros_like(dq)
+    tm.tm_triangle_attn_fwd_ws(zq, dk, dv, o, wl.B, wl.Hq, wl.Hkv, wl.N, wl.D, wl.scale, wl.S,
+                               wl.W, wl.L, ws, n)
+    torch.cuda.synchronize()
+    vf = I.bf16_bits_to_f32(v).astype(np.float64)
+    pre = np.concatenate([np.zeros_like(vf[:, :1]), np.cumsum(vf, axis=1)], axis=1)
+    G = wl.Hq // wl.Hkv
+    worst = 0.0
+    for r0 in range(0, wl.N, 16384):
+        rr = np.arange(r0, min(wl.N, r0 + 16384))
+        got = from_dev(o[:, r0:r0 + len(rr)]).reshape(wl.B, len(rr), wl.Hkv, G, wl.D)
+        want = zero_query_expected(vf, pre, wl.N, wl.S, wl.W, wl.L, rr)[:, :, :, None, :]
+        assert np.isfinite(got).all()
+        worst = max(worst, float(np.abs(got - want).max()))
+    assert worst <= 2e-2, worst
