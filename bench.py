@@ -63,6 +63,16 @@ def load_peaks():
         return {"burst": 1590.0, "sustained": 1400.0, "hbm": 6650.0, "source": "fallback"}
 
 
+def workload_config(wl, W, n_ranks) -> dict:
+    """The `config` object of both arms' JSON lines (same workload, same keys)."""
+    q_gb = wl.B * wl.N * wl.Hq * wl.D * 2 / 1e9
+    return {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "N": wl.N, "D": wl.D,
+            "S": wl.S, "W": W, "L": wl.L, "tri_start": wl.tri_start,
+            "step": "triangle layer + causal layer via tm_trianglemix_attn_fwd_ws",
+            "l2": "inputs larger than L2 (q alone is %.2f GB)" % q_gb,
+            "parallelism": "replicas" if n_ranks > 1 else "single"}
+
+
 def tile_flop(wl, causal, W=None) -> float:
     import long_context_prefill_trianglemix_b200 as tm
     tiles = tm.tm_kept_tiles(wl.N, causal, wl.S, wl.W if W is None else W, wl.L)
@@ -196,8 +206,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "N": wl.N,
-                   "D": wl.D, "S": wl.S, "W": W, "L": wl.L},
+        "config": workload_config(wl, W, ws),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -389,12 +398,7 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "N": wl.N,
-                   "D": wl.D, "S": wl.S, "W": W, "L": wl.L, "tri_start": wl.tri_start,
-                   "step": "triangle layer + causal layer via tm_trianglemix_attn_fwd_ws",
-                   "split_workspace_bytes": ws_bytes,
-                   "l2": "inputs larger than L2 (q alone is %.2f GB)" % (dq.numel() * 2 / 1e9),
-                   "parallelism": "replicas" if ws > 1 else "single"},
+        "config": dict(workload_config(wl, W, ws), split_workspace_bytes=ws_bytes),
         "triangle_ms": tri_avg,
         "triangle_ms_p10_p90": [float(np.percentile(tri_ms, 10)), float(np.percentile(tri_ms, 90))],
         "causal_ms": sum(cau_ms) / args.steps,
