@@ -194,11 +194,14 @@ __host__ __device__ __forceinline__ int big_count(const AttnParams& p, int c, in
 // Normal index (counted from 0 after the big items) of CTA c's j-th normal item.
 __host__ __device__ __forceinline__ long long normal_index(const AttnParams& p, int c, int g, int j) {
   const int ga = g - p.n_a;
-  if (c >= p.n_a) {
-    if (j < p.n_skip) return static_cast<long long>(c - p.n_a) + static_cast<long long>(j) * ga;
-    return static_cast<long long>(p.n_skip) * ga + static_cast<long long>(j - p.n_skip) * g + c;
-  }
-  return static_cast<long long>(p.n_skip) * ga + static_cast<long long>(j) * g + c;
+  if (c >= p.n_a && j < p.n_skip)
+    return static_cast<long long>(c - p.n_a) + static_cast<long long>(j) * ga;
+  // main rounds r = 0, 1, ...: odd rounds are dealt in reverse CTA order, so a
+  // CTA that drew a long item of its round draws a short one next and the
+  // CTAs' positions in the tile streams do not drift apart
+  const int r = c >= p.n_a ? j - p.n_skip : j;
+  return static_cast<long long>(p.n_skip) * ga + static_cast<long long>(r) * g +
+         ((r & 1) ? g - 1 - c : c);
 }
 
 __host__ __device__ __forceinline__ int work_count(const AttnParams& p, int c, int g) {
@@ -343,6 +346,9 @@ struct WorkCursor {
   int d_pr, d_kvh, d_b, d_qi;       // digits of the current stride
   int rot, d_rot;                   // qi * pair_rot and d_qi * pair_rot, mod npairs
   int krot, d_krot;                 // qi * kv_rot and d_qi * kv_rot, mod Hkv
+  // main rounds alternate two strides (odd rounds run in reverse CTA order)
+  int e_pr, e_kvh, e_b, e_qi, e_rot, e_krot;  // digits of the other stride
+  int flip;                                  // 1: the strides alternate
   __host__ __device__ __forceinline__ void set_item(const AttnParams& p, long long item) {
     qi = static_cast<int>(item / p.units);
     const int u = static_cast<int>(item - static_cast<long long>(qi) * p.units);
@@ -366,8 +372,16 @@ struct WorkCursor {
   __host__ __device__ __forceinline__ void enter_phase(const AttnParams& p) {
     set_item(p, p.n_hunits + normal_index(p, c, g, j));
     const bool late = c >= p.n_a && j < p.n_skip;
-    set_stride(p, late ? g - p.n_a : g);
     phase_end = late ? p.n_skip : 0x7fffffff;
+    flip = late ? 0 : 1;
+    if (late) {
+      set_stride(p, g - p.n_a);
+      return;
+    }
+    // the main phase starts at round 0 (even): first 2g - 1 - 2c, then 2c + 1
+    set_stride(p, 2 * c + 1);
+    e_pr = d_pr; e_kvh = d_kvh; e_b = d_b; e_qi = d_qi; e_rot = d_rot; e_krot = d_krot;
+    set_stride(p, 2 * g - 1 - 2 * c);
   }
   __host__ __device__ __forceinline__ void init(const AttnParams& p, int cta, int grid) {
     c = cta;
@@ -419,6 +433,14 @@ struct WorkCursor {
         krot += d_krot + (carry ? p.kv_rot : 0);  // < 3 Hkv
         if (krot >= p.Hkv) krot -= p.Hkv;
         if (krot >= p.Hkv) krot -= p.Hkv;
+        if (flip) {  // swap to the other stride for the next step
+          int t0 = d_pr; d_pr = e_pr; e_pr = t0;
+          t0 = d_kvh; d_kvh = e_kvh; e_kvh = t0;
+          t0 = d_b; d_b = e_b; e_b = t0;
+          t0 = d_qi; d_qi = e_qi; e_qi = t0;
+          t0 = d_rot; d_rot = e_rot; e_rot = t0;
+          t0 = d_krot; d_krot = e_krot; e_krot = t0;
+        }
       }
     }
     ++k;
