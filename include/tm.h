@@ -305,6 +305,20 @@ TM_API int tm_debug_schedule(int B, int Hq, int Hkv, int N, int causal, int S, i
                              int num_ctas, int split, int* out, long long cap, long long* count);
 
 /*
+ * Failure-detection check (tests only): runs tm_triangle_attn_fwd with one
+ * fault injected on the host side of the pipeline — the producer of CTA 0
+ * delivers no Q tile for its first item and stops. That CTA's MMA issuer then
+ * gives up on its bounded wait (about two seconds), records TM_ERR_TIMEOUT in
+ * the device status word, and all of the CTA's roles leave, drain their copies
+ * and free TMEM; the other CTAs finish. o is left partly unwritten. The call
+ * itself returns TM_OK (or an argument error); tm_get_device_status then
+ * reports TM_ERR_TIMEOUT, and the context stays usable.
+ */
+TM_API int tm_debug_inject_stall(const void* q, const void* k, const void* v, void* o, int B,
+                                 int Hq, int Hkv, int N, int D, float scale, int S, int W, int L,
+                                 void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word of the
  * current device: TM_OK, or TM_ERR_TIMEOUT if a kernel gave up on a wait
  * since the last call. TM_ERR_CUDA if the synchronisation itself failed.

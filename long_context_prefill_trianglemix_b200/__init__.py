@@ -30,6 +30,7 @@ EXPORTED = (
     "tm_trianglemix_attn_fwd_ws", "tm_trianglemix_attn_fwd_noalloc", "tm_block_sparse_attn_fwd",
     "tm_trianglemix_sparse_attn_fwd", "tm_flashprefill_workspace_size",
     "tm_flashprefill_index_capacity", "tm_flashprefill_block_index", "tm_triangle_attn_fwd_heads",
+    "tm_debug_inject_stall",
 )
 
 
@@ -86,6 +87,7 @@ def lib() -> ctypes.CDLL:
             "tm_flashprefill_block_index": (ci, [vp, vp, ci, ci, ci, ci, ci, cf, cf, ci, vp, cll,
                                                  vp, vp, cll, vp, vp]),
             "tm_get_device_status": (ci, [vp]),
+            "tm_debug_inject_stall": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci, ci, vp]),
             "tm_status_string": (ctypes.c_char_p, [ci]),
         }
         for name, (res, args) in sig.items():
@@ -280,6 +282,11 @@ def tm_debug_schedule(B, Hq, Hkv, N, causal, S, W, L, num_ctas=148, split=False,
                                                         num_ctas, int(split), out.ctypes.data,
                                                         cnt.value, ctypes.byref(cnt)))
     return out[: cnt.value]
+
+
+def tm_debug_inject_stall(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L, stream=None):
+    return _check("tm_debug_inject_stall", lib().tm_debug_inject_stall(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, Hkv, N, D, scale, S, W, L, _stream(stream)))
 
 
 def tm_get_device_status(stream=None) -> int:

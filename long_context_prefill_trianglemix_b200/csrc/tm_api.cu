@@ -89,10 +89,11 @@ int scratch_address(void** out) {
 int run(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv, int N, int D,
         float scale, const trimix::Pattern& pat, void* ws, long long ws_bytes, void* stream,
         const int* bs_off = nullptr, const int* bs_idx = nullptr, long long bs_nnz = 0,
-        const int* hS = nullptr, const int* hW = nullptr) {
+        const int* hS = nullptr, const int* hW = nullptr, int inject_cta = -1) {
   trimix::LaunchArgs a;
   a.hS = hS;
   a.hW = hW;
+  a.inject_cta = inject_cta;
   a.bs_off = bs_off;
   a.bs_idx = bs_idx;
   a.bs_nnz = bs_nnz;
@@ -392,6 +393,15 @@ TM_API int tm_debug_schedule(int B, int Hq, int Hkv, int N, int causal, int S, i
     return TM_ERR_INVALID_ARG;
   return trimix::debug_schedule(B, Hq, Hkv, N, trimix::make_pattern(N, causal, S, W, L), num_ctas,
                                 split, out, cap, count);
+}
+
+TM_API int tm_debug_inject_stall(const void* q, const void* k, const void* v, void* o, int B,
+                                 int Hq, int Hkv, int N, int D, float scale, int S, int W, int L,
+                                 void* stream) {
+  if (int rc = validate_common(q, k, v, o, B, Hq, Hkv, N, D, scale)) return rc;
+  if (int rc = validate_pattern(S, W, L)) return rc;
+  return run(q, k, v, o, B, Hq, Hkv, N, D, scale, trimix::make_pattern(N, 0, S, W, L), nullptr, 0,
+             stream, nullptr, nullptr, 0, nullptr, nullptr, /*inject_cta=*/0);
 }
 
 TM_API int tm_get_device_status(void* stream) { return trimix::read_and_clear_device_status(stream); }

@@ -163,6 +163,10 @@ struct AttnParams {
   // kv_rot rotates the kv head the same way (per-head band launches, whose kv
   // heads differ in cost); it permutes whole groups, which stay adjacent too.
   int pair_rot, kv_rot;
+  // Test hook (-1 in every product launch): the producer of this CTA delivers
+  // no Q for its first item and leaves, so the issuer's bounded wait on q_full
+  // runs out; the CTA records a timeout and every role exits cleanly.
+  int inject_cta;
   // Split pieces (nsplit > 1): each writes its unnormalised partial (O, running
   // max m, sum l) of every 32-row warp slice to ws_rec and counts itself in
   // ws_cnt (one counter per cut item, Q tile and warp, zero at launch); the
@@ -566,6 +570,10 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, Bars<Cfg<D>::
     const int t_end = imin(bt.count(), it.t1);
     if (t_end <= it.t0) continue;  // an empty block-sparse list: nothing to load
     if (!(ok = load_kv(it, bt, it.t0))) break;
+    if (p.inject_cta == static_cast<int>(blockIdx.x) && it_cnt == 0) {
+      ok = false;  // test hook: no Q for the first item (drained and left below)
+      break;
+    }
     if (!(ok = wait_bar(&bars->q_empty, (it_cnt & 1u) ^ 1u, abort_flag, kSiteQEmpty))) break;
     bars->item_T = t_end - it.t0;
     bars->item_v1 = it.v1;
@@ -1268,6 +1276,7 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
   p->ws_cnt = nullptr;
   p->pair_rot = 0;
   p->kv_rot = 0;
+  p->inject_cta = -1;
   p->bs_off = nullptr;
   p->bs_idx = nullptr;
   p->bs_nnz = 0;
@@ -1408,6 +1417,7 @@ int launch_attention_d(const LaunchArgs& a, DeviceInfo* di) {
   const int grid = build_schedule(a.B, a.Hq, a.Hkv, a.N, a.pat, di->sms, a.ws != nullptr, &p,
                                   sparse, a.hS != nullptr);
   p.sl2 = a.scale * 1.4426950408889634f;
+  p.inject_cta = a.inject_cta;
   if (a.hS) {  // per-head bands; a.pat already holds the maxima
     if (a.Hq > kMaxBandHeads) return TM_ERR_UNSUPPORTED;
     p.ph = 1;

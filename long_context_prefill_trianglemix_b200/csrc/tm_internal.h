@@ -26,6 +26,7 @@ struct LaunchArgs {
   long long bs_nnz;
   const int* hS;      // per-head sinks and windows (host, Hq each), or nullptr
   const int* hW;
+  int inject_cta;     // test hook: -1, or the CTA whose first Q is never delivered
   void* stream;
 };
 

@@ -200,3 +200,9 @@ def test_seeded_head_bands():
     assert len(set(W.tolist())) > 20
     S2, W2 = I.head_bands(32, 0)
     assert np.array_equal(S, S2) and np.array_equal(W, W2)
+
+
+def test_inject_stall_validates_before_launch():
+    args = (FAKE, FAKE, FAKE, FAKE + 0x100000, 1, 4, 4, 64, 64, 0.1)
+    assert tm.lib().tm_debug_inject_stall(*args, 4, 0, 2, None) == tm.TM_ERR_INVALID_ARG
+    assert tm.lib().tm_debug_inject_stall(0, *args[1:], 4, 8, 2, None) == tm.TM_ERR_INVALID_ARG
