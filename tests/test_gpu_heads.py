@@ -108,3 +108,18 @@ def test_tp8_shard_128k_bands_with_split_sampled_rows():
     want = oracle.attention_heads(q, k, v, wl.B, wl.Hq, wl.Hkv, wl.N, wl.D, wl.scale, Sh, Wh,
                                   wl.L, rows=rows)
     assert_close(from_dev(o[:, torch.tensor(rows, device="cuda")]), want, "tp8 128K bands")
+
+
+def test_llama_128k_bench_bands_sampled_rows():
+    """The bench's per-head leg: all 32 q heads of the 128K Llama-3-8B shape with
+    the seeded bands (windows 512..4096, sinks {0, 64}), sampled rows."""
+    import torch
+    wl = I.WORKLOADS["llama3-8b-128k"]
+    q, k, v = I.make_qkv(wl, wl.tri_start)
+    Sh, Wh = I.head_bands(wl.Hq, 0)
+    o = run_heads(to_dev(q), to_dev(k), to_dev(v), wl.B, wl.Hq, wl.Hkv, wl.N, wl.D, wl.scale,
+                  Sh, Wh, wl.L)
+    rows = sample_rows(wl.N, wl.L, 14, 32, 64, n_last=32)
+    want = oracle.attention_heads(q, k, v, wl.B, wl.Hq, wl.Hkv, wl.N, wl.D, wl.scale, Sh, Wh,
+                                  wl.L, rows=rows)
+    assert_close(from_dev(o[:, torch.tensor(rows, device="cuda")]), want, "llama 128K bands")
