@@ -40,6 +40,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <mutex>
@@ -1205,18 +1206,36 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// Per-device facts. ready / supported / sms are written once under g_mutex and
+// read by callers that went through device_info (which takes it); the
+// per-kernel "shared-memory attribute set" flags are atomics, set under
+// g_mutex after the attribute call and read without it.
 struct DeviceInfo {
   bool ready = false;
   bool supported = false;
   int sms = 0;
-  bool attr_set[2] = {false, false};
-  bool probe_attr_set[2] = {false, false};
-  bool disc_attr_set[2] = {false, false};
+  std::atomic<bool> attr_set[2] = {false, false};
+  std::atomic<bool> probe_attr_set[2] = {false, false};
+  std::atomic<bool> disc_attr_set[2] = {false, false};
 };
 
+constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
 EncodeTiledFn g_encode = nullptr;
-std::vector<DeviceInfo> g_devices;
+DeviceInfo g_devices[kMaxDevices];  // fixed: pointers handed out stay valid
+
+// Sets a kernel's dynamic shared-memory limit once per device.
+template <class K>
+int set_smem_once(std::atomic<bool>& flag, K kernel, int bytes) {
+  if (flag.load(std::memory_order_acquire)) return TM_OK;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (flag.load(std::memory_order_relaxed)) return TM_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return TM_ERR_CUDA;
+  flag.store(true, std::memory_order_release);
+  return TM_OK;
+}
 
 int get_encode_fn() {
   if (g_encode) return TM_OK;
@@ -1233,9 +1252,9 @@ int get_encode_fn() {
 int device_info(DeviceInfo** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return TM_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return TM_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mutex);
   if (int rc = get_encode_fn()) return rc;
-  if (static_cast<int>(g_devices.size()) <= dev) g_devices.resize(dev + 1);
   DeviceInfo& di = g_devices[dev];
   if (!di.ready) {
     cudaDeviceProp prop;
@@ -1390,8 +1409,7 @@ WsLayout ws_layout(const AttnParams& p, int D) {
 template <int D>
 int launch_attention_d(const LaunchArgs& a, DeviceInfo* di) {
   const int kidx = D == 128 ? 1 : 0;
-  if (!di->attr_set[kidx]) {
-    std::lock_guard<std::mutex> lock(g_mutex);
+  if (!di->attr_set[kidx].load(std::memory_order_acquire)) {
     // setmaxnreg redistributes exactly kThreads x kLaunchRegs registers; any
     // other launch register count could leave the increase waiting forever.
     cudaFuncAttributes fa;
@@ -1401,10 +1419,7 @@ int launch_attention_d(const LaunchArgs& a, DeviceInfo* di) {
               kLaunchRegs);
       return TM_ERR_UNSUPPORTED;
     }
-    if (cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg<D>::kSmemBytes) != cudaSuccess)
-      return TM_ERR_CUDA;
-    di->attr_set[kidx] = true;
+    if (int rc = set_smem_once(di->attr_set[kidx], attn_kernel<D>, Cfg<D>::kSmemBytes)) return rc;
   }
   CUtensorMap tq, tk, tv, to;
   if (encode_bnhd(&tq, a.q, a.B, a.N, a.Hq, D, BM) || encode_bnhd(&tk, a.k, a.B, a.N, a.Hkv, D, BN) ||
@@ -1486,13 +1501,8 @@ DiscLayout disc_layout(int B, int Hkv, int N, int D, int R) {
 template <int D>
 int launch_discovery_d(const DiscArgs& a, DeviceInfo* di) {
   const int kidx = D == 128 ? 1 : 0;
-  if (!di->disc_attr_set[kidx]) {
-    std::lock_guard<std::mutex> lock(g_mutex);
-    if (cudaFuncSetAttribute(score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             DiscCfg<D>::kSmem) != cudaSuccess)
-      return TM_ERR_CUDA;
-    di->disc_attr_set[kidx] = true;
-  }
+  if (int rc = set_smem_once(di->disc_attr_set[kidx], score_kernel<D>, DiscCfg<D>::kSmem))
+    return rc;
   const int G = a.Hq / a.Hkv, R = G * a.P, nqb = (a.N + BM - 1) / BM;
   const DiscLayout l = disc_layout(a.B, a.Hkv, a.N, D, R);
   if (a.ws_bytes < l.total) return TM_ERR_INVALID_ARG;
@@ -1607,12 +1617,7 @@ static int launch_probe_d(const void* q, const void* k, const void* v, float* s_
                           void* stream, DeviceInfo* di) {
   const int kidx = D == 128 ? 1 : 0;
   const int smem = 3 * Cfg<D>::kTileBytes + 64 + 1024;
-  if (!di->probe_attr_set[kidx]) {
-    if (cudaFuncSetAttribute(mma_probe_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
-      return TM_ERR_CUDA;
-    di->probe_attr_set[kidx] = true;
-  }
+  if (int rc = set_smem_once(di->probe_attr_set[kidx], mma_probe_kernel<D>, smem)) return rc;
   CUtensorMap tq, tk, tv;
   if (encode_bnhd(&tq, q, 1, 128, 1, D, 128) || encode_bnhd(&tk, k, 1, 128, 1, D, 128) ||
       encode_bnhd(&tv, v, 1, 128, 1, D, 128))
