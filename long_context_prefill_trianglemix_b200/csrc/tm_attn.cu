@@ -620,6 +620,12 @@ template <int D>
 __device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStages>* bars,
                                          uint8_t* smem, uint32_t tmem_base) {
   constexpr int NST = Cfg<D>::kStages;
+  // The whole warp runs this loop in step (waits, counters, descriptors), and
+  // one lane, elected once, issues every MMA and commit: a commit tracks only
+  // the MMAs of the thread that issues it. Keeping the warp converged lets the
+  // operands live in uniform registers, so an MMA costs few issue slots on a
+  // sub-partition that two softmax warps keep busy.
+  const bool leader = elect_one();
   volatile int* abort_flag = &bars->abort_flag;
   const uint32_t q0 = desc_lo_sw128(smem_addr(smem), 16), q1 = desc_lo_sw128(smem_addr(smem) + Cfg<D>::kTileBytes, 16);
   const uint32_t ring = smem_addr(smem + Cfg<D>::kRingOff);
@@ -630,13 +636,14 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStag
   const uint32_t tO0 = tmem_base + Cfg<D>::kTmemO0, tO1 = tmem_base + Cfg<D>::kTmemO1;
   uint32_t kv_cnt = 0, it_cnt = 0, pc0 = 0, pc1 = 0, oe0 = 0, oe1 = 0;
   bool ok = true;
-#define TM_WAIT(bar, par, site)                                      \
-  if (!(ok = wait_bar((bar), (par), abort_flag, (site)))) break; \
+#define TM_WAIT(bar, par, site)                                                            \
+  if (!(ok = __all_sync(0xffffffffu, wait_bar((bar), (par), abort_flag, (site))))) break; \
   tc_fence_after();
   // Items come from the producer's descriptors (no work cursor here: the
   // issuer's registers are few and its loop is on the critical path).
-  if (!(ok = wait_bar(&bars->q_full, it_cnt & 1u, abort_flag, kSiteQFull))) {
-    mma_commit(&bars->mma_done);
+  if (!(ok = __all_sync(0xffffffffu, wait_bar(&bars->q_full, it_cnt & 1u, abort_flag, kSiteQFull)))) {
+    if (leader) mma_commit(&bars->mma_done);
+    __syncwarp();
     drain_wait(&bars->mma_done, 0);
     return;
   }
@@ -650,14 +657,20 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStag
     if (!started) {
       kst = kv_cnt % NST;
       TM_WAIT(&bars->kv_full[kst], (kv_cnt / NST) & 1u, kSiteKvFull);
-      issue_qk<D>(tS0, q0, k_lo0 + kst * kStageLo);
-      mma_commit(&bars->s_full[0]);
+      if (leader) issue_qk<D>(tS0, q0, k_lo0 + kst * kStageLo);
+      __syncwarp();
+      if (leader) mma_commit(&bars->s_full[0]);
+      __syncwarp();
       if (v1) {
-        issue_qk<D>(tS1, q1, k_lo0 + kst * kStageLo);
-        mma_commit(&bars->s_full[1]);
+        if (leader) issue_qk<D>(tS1, q1, k_lo0 + kst * kStageLo);
+        __syncwarp();
+        if (leader) mma_commit(&bars->s_full[1]);
+        __syncwarp();
       }
-      if (T == 1) mma_commit(&bars->q_empty);
-      mma_commit(&bars->kv_empty[kst]);
+      if (T == 1 && leader) mma_commit(&bars->q_empty);
+      __syncwarp();
+      if (leader) mma_commit(&bars->kv_empty[kst]);
+      __syncwarp();
       ++kv_cnt;
     }
     int Tn = 0;
@@ -671,35 +684,47 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStag
         ++oe0;
       }
       TM_WAIT(&bars->p_full[0], pc0 & 1u, kSitePFull);
-      issue_pv<D, 0, 4>(tO0, tS0, v_lo0 + vst * kStageLo, t > 0 ? 1u : 0u);
+      if (leader) issue_pv<D, 0, 4>(tO0, tS0, v_lo0 + vst * kStageLo, t > 0 ? 1u : 0u);
+      __syncwarp();
       TM_WAIT(&bars->p_full[1], pc0 & 1u, kSitePFull);
       ++pc0;
-      issue_pv<D, 4, 8>(tO0, tS0, v_lo0 + vst * kStageLo, 1u);
+      if (leader) issue_pv<D, 4, 8>(tO0, tS0, v_lo0 + vst * kStageLo, 1u);
+      __syncwarp();
       const uint32_t kidx = kv_cnt + 1;
       kst = kidx % NST;
       TM_WAIT(&bars->kv_full[kst], (kidx / NST) & 1u, kSiteKvFull);
-      issue_qk<D>(tS0, q0, k_lo0 + kst * kStageLo);
-      mma_commit(&bars->s_full[0]);
-      if (!v1 && t + 1 == T - 1) mma_commit(&bars->q_empty);
+      if (leader) issue_qk<D>(tS0, q0, k_lo0 + kst * kStageLo);
+      __syncwarp();
+      if (leader) mma_commit(&bars->s_full[0]);
+      __syncwarp();
+      if (!v1 && t + 1 == T - 1 && leader) mma_commit(&bars->q_empty);
+      __syncwarp();
       if (v1) {
         if (t == 0) {
           TM_WAIT(&bars->o_empty[1], (oe1 & 1u) ^ 1u, kSiteOEmpty);
           ++oe1;
         }
         TM_WAIT(&bars->p_full[2], pc1 & 1u, kSitePFull);
-        issue_pv<D, 0, 4>(tO1, tS1, v_lo0 + vst * kStageLo, t > 0 ? 1u : 0u);
+        if (leader) issue_pv<D, 0, 4>(tO1, tS1, v_lo0 + vst * kStageLo, t > 0 ? 1u : 0u);
+        __syncwarp();
         TM_WAIT(&bars->p_full[3], pc1 & 1u, kSitePFull);
         ++pc1;
-        issue_pv<D, 4, 8>(tO1, tS1, v_lo0 + vst * kStageLo, 1u);
+        if (leader) issue_pv<D, 4, 8>(tO1, tS1, v_lo0 + vst * kStageLo, 1u);
+        __syncwarp();
       }
-      mma_commit(&bars->kv_empty[vst]);  // V_t free once both P.V products are done
+      if (leader) mma_commit(&bars->kv_empty[vst]);  // V_t free once both P.V products are done
+      __syncwarp();
       ++kv_cnt;
       if (v1) {
-        issue_qk<D>(tS1, q1, k_lo0 + kst * kStageLo);
-        mma_commit(&bars->s_full[1]);
-        if (t + 1 == T - 1) mma_commit(&bars->q_empty);
+        if (leader) issue_qk<D>(tS1, q1, k_lo0 + kst * kStageLo);
+        __syncwarp();
+        if (leader) mma_commit(&bars->s_full[1]);
+        __syncwarp();
+        if (t + 1 == T - 1 && leader) mma_commit(&bars->q_empty);
+        __syncwarp();
       }
-      mma_commit(&bars->kv_empty[kst]);  // K_{t+1} free once both Q.K products are done
+      if (leader) mma_commit(&bars->kv_empty[kst]);  // K_{t+1} free once both Q.K products are done
+      __syncwarp();
       ++kv_cnt;
     }
     if (!ok) break;
@@ -713,11 +738,14 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStag
         ++oe0;
       }
       TM_WAIT(&bars->p_full[0], pc0 & 1u, kSitePFull);
-      issue_pv<D, 0, 4>(tO0, tS0, v_lo0 + vst * kStageLo, t > 0 ? 1u : 0u);
+      if (leader) issue_pv<D, 0, 4>(tO0, tS0, v_lo0 + vst * kStageLo, t > 0 ? 1u : 0u);
+      __syncwarp();
       TM_WAIT(&bars->p_full[1], pc0 & 1u, kSitePFull);
       ++pc0;
-      issue_pv<D, 4, 8>(tO0, tS0, v_lo0 + vst * kStageLo, 1u);
-      mma_commit(&bars->o_full[0]);
+      if (leader) issue_pv<D, 4, 8>(tO0, tS0, v_lo0 + vst * kStageLo, 1u);
+      __syncwarp();
+      if (leader) mma_commit(&bars->o_full[0]);
+      __syncwarp();
       // the next item's descriptor (and Q), then its S0
       TM_WAIT(&bars->q_full, it_cnt & 1u, kSiteQFull);
       ++it_cnt;
@@ -727,9 +755,12 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStag
         const uint32_t kidx = kv_cnt + 1;
         kst = kidx % NST;
         TM_WAIT(&bars->kv_full[kst], (kidx / NST) & 1u, kSiteKvFull);
-        issue_qk<D>(tS0, q0, k_lo0 + kst * kStageLo);
-        mma_commit(&bars->s_full[0]);
-        if (!v1n && Tn == 1) mma_commit(&bars->q_empty);
+        if (leader) issue_qk<D>(tS0, q0, k_lo0 + kst * kStageLo);
+        __syncwarp();
+        if (leader) mma_commit(&bars->s_full[0]);
+        __syncwarp();
+        if (!v1n && Tn == 1 && leader) mma_commit(&bars->q_empty);
+        __syncwarp();
       }
       if (v1) {
         if (t == 0) {
@@ -737,21 +768,29 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStag
           ++oe1;
         }
         TM_WAIT(&bars->p_full[2], pc1 & 1u, kSitePFull);
-        issue_pv<D, 0, 4>(tO1, tS1, v_lo0 + vst * kStageLo, t > 0 ? 1u : 0u);
+        if (leader) issue_pv<D, 0, 4>(tO1, tS1, v_lo0 + vst * kStageLo, t > 0 ? 1u : 0u);
+        __syncwarp();
         TM_WAIT(&bars->p_full[3], pc1 & 1u, kSitePFull);
         ++pc1;
-        issue_pv<D, 4, 8>(tO1, tS1, v_lo0 + vst * kStageLo, 1u);
-        mma_commit(&bars->o_full[1]);
+        if (leader) issue_pv<D, 4, 8>(tO1, tS1, v_lo0 + vst * kStageLo, 1u);
+        __syncwarp();
+        if (leader) mma_commit(&bars->o_full[1]);
+        __syncwarp();
       }
-      mma_commit(&bars->kv_empty[vst]);
+      if (leader) mma_commit(&bars->kv_empty[vst]);
+      __syncwarp();
       ++kv_cnt;
       if (Tn > 0) {
         if (v1n) {
-          issue_qk<D>(tS1, q1, k_lo0 + kst * kStageLo);
-          mma_commit(&bars->s_full[1]);
-          if (Tn == 1) mma_commit(&bars->q_empty);
+          if (leader) issue_qk<D>(tS1, q1, k_lo0 + kst * kStageLo);
+          __syncwarp();
+          if (leader) mma_commit(&bars->s_full[1]);
+          __syncwarp();
+          if (Tn == 1 && leader) mma_commit(&bars->q_empty);
+          __syncwarp();
         }
-        mma_commit(&bars->kv_empty[kst]);
+        if (leader) mma_commit(&bars->kv_empty[kst]);
+        __syncwarp();
         ++kv_cnt;
       }
     } while (false);
@@ -762,7 +801,8 @@ __device__ __forceinline__ void mma_role(const AttnParams& p, Bars<Cfg<D>::kStag
   }
 #undef TM_WAIT
   // Every MMA issued above must finish before TMEM is released.
-  mma_commit(&bars->mma_done);
+  if (leader) mma_commit(&bars->mma_done);
+  __syncwarp();
   drain_wait(&bars->mma_done, 0);
 }
 
@@ -1069,7 +1109,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) producer_role<D>(p, bars, smem, &tq, &tk, &tv);
     __syncwarp();
   } else if (warp == kWarpMma) {
-    if (lane == 0) mma_role<D>(p, bars, smem, tmem_base);
+    mma_role<D>(p, bars, smem, tmem_base);
     __syncwarp();
   }
   tc_fence_before();
