@@ -40,7 +40,7 @@ BM = BN = 128
 # triangle launch of the default workload (llama3-8b-128k, W=2048) from one ncu
 # capture of this bench command, keyed by the hash of the kernel sources it was
 # taken on; reported only while the sources still match (else null).
-TRAFFIC = {"d0d067a0eb5b540f": 2.273e9 + 1.043e9}
+TRAFFIC = {"a9e9800ed9a867ac": 2.200e9 + 1.040e9}
 
 
 def kernel_source_hash() -> str:

@@ -9,6 +9,7 @@ cross-compiles sm_100a without a GPU.
 from __future__ import annotations
 
 import glob
+import hashlib
 import os
 import shutil
 import subprocess
@@ -30,18 +31,40 @@ def _nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def _stale(target: str, sources) -> bool:
-    if not os.path.exists(target):
+def _stamp(sources, cmd) -> str:
+    """Digest of the build command and of every source file's path and bytes."""
+    h = hashlib.sha256()
+    h.update("\0".join(cmd).encode())
+    for s in sorted(sources):
+        h.update(os.path.relpath(s, ROOT).encode())
+        with open(s, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def _stale(target: str, sources, cmd) -> bool:
+    """A library is rebuilt unless its stamp file holds the digest of the
+    sources and command it would be built from now. File times are not used:
+    a copied tree can leave a library that is older than its sources looking
+    newer (or the reverse)."""
+    if not os.path.exists(target) or not os.path.exists(target + ".stamp"):
         return True
-    t = os.path.getmtime(target)
-    return any(os.path.getmtime(s) > t for s in sources)
+    with open(target + ".stamp") as f:
+        return f.read().strip() != _stamp(sources, cmd)
+
+
+def _write_stamp(target: str, sources, cmd) -> None:
+    with open(target + ".stamp", "w") as f:
+        f.write(_stamp(sources, cmd) + "\n")
 
 
 def build_inputs(force: bool = False) -> str:
     src = os.path.join(PKG, "inputs", "tm_inputs.c")
-    if force or _stale(LIBINPUTS, [src]):
-        subprocess.run(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread", src, "-lm",
-                        "-o", LIBINPUTS], check=True)
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread", src, "-lm", "-o", LIBINPUTS]
+    key = [c if c not in (src, LIBINPUTS) else os.path.relpath(c, ROOT) for c in cmd]
+    if force or _stale(LIBINPUTS, [src], key):
+        subprocess.run(cmd, check=True)
+        _write_stamp(LIBINPUTS, [src], key)
     return LIBINPUTS
 
 
@@ -49,20 +72,28 @@ def cuda_sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def build_lib(force: bool = False, verbose_ptxas: bool = False, extra=()) -> str:
+def lib_inputs(extra=()):
+    """(CUDA sources, every file the library depends on, nvcc flags)."""
     srcs = cuda_sources()
     deps = srcs + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
+    flags = [*extra, *NVCC_ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared",
+             "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden"]
+    return srcs, deps, flags
+
+
+def build_lib(force: bool = False, verbose_ptxas: bool = False, extra=()) -> str:
+    srcs, deps, flags = lib_inputs(extra)
     if not srcs:
         raise RuntimeError("no CUDA sources")
-    if not (force or _stale(LIBTM, deps)):
+    if not (force or verbose_ptxas or _stale(LIBTM, deps, flags)):
         return LIBTM
-    cmd = [_nvcc(), *NVCC_ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared",
-           "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
-           "-I", INCLUDE, "-I", CSRC, *srcs, "-o", LIBTM]
+    cmd = [_nvcc(), *flags, "-I", INCLUDE, "-I", CSRC, *srcs, "-o", LIBTM]
     if verbose_ptxas:
         cmd.insert(1, "-Xptxas=-v")
-    cmd[1:1] = list(extra)
+    if os.path.exists(LIBTM + ".stamp"):
+        os.remove(LIBTM + ".stamp")  # no stamp while the library is being replaced
     subprocess.run(cmd, check=True)
+    _write_stamp(LIBTM, deps, flags)
     return LIBTM
 
 
