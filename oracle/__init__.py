@@ -8,6 +8,7 @@ input generator, which holds no attention arithmetic.
 from __future__ import annotations
 
 import ctypes
+import hashlib
 import os
 import subprocess
 
@@ -19,11 +20,19 @@ _lib = None
 
 
 def build(force: bool = False) -> str:
-    """Compile ``liboracle.so`` with the host C++ compiler (no CUDA)."""
+    """Compile ``liboracle.so`` with the host C++ compiler (no CUDA). It is
+    rebuilt unless ``liboracle.so.stamp`` holds the SHA-256 of the compiler
+    flags and the source (file times are not trusted across copies)."""
     src = os.path.join(_HERE, "tm_oracle.cpp")
-    if force or not os.path.exists(LIB_PATH) or os.path.getmtime(LIB_PATH) < os.path.getmtime(src):
-        cmd = ["g++", "-O2", "-std=c++17", "-fPIC", "-shared", "-pthread", src, "-o", LIB_PATH]
-        subprocess.run(cmd, check=True)
+    flags = ["-O2", "-std=c++17", "-fPIC", "-shared", "-pthread"]
+    with open(src, "rb") as f:
+        digest = hashlib.sha256((" ".join(flags) + "\n").encode() + f.read()).hexdigest()
+    stamp = LIB_PATH + ".stamp"
+    fresh = os.path.exists(LIB_PATH) and os.path.exists(stamp) and open(stamp).read().strip() == digest
+    if force or not fresh:
+        subprocess.run(["g++", *flags, src, "-o", LIB_PATH], check=True)
+        with open(stamp, "w") as f:
+            f.write(digest + "\n")
     return LIB_PATH
 
 
