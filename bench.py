@@ -40,7 +40,7 @@ BM = BN = 128
 # triangle launch of the default workload (llama3-8b-128k, W=2048) from one ncu
 # capture of this bench command, keyed by the hash of the kernel sources it was
 # taken on; reported only while the sources still match (else null).
-TRAFFIC = {"a9e9800ed9a867ac": 2.200e9 + 1.040e9}
+TRAFFIC = {"8f8da125031ac4bf": 2.354e9 + 1.042e9}
 
 
 def kernel_source_hash() -> str:
@@ -289,16 +289,20 @@ def run_ours(args):
     total_ms = ev[0][0].elapsed_time(ev[-1][2])
     tri_sum = sum(tri_ms)
 
-    # end to end through the same call: pinned host -> device, layer, device -> host
+    # end to end through the host-buffer call: pinned host q, k, v in, the
+    # triangle layer, pinned host o out, streamed in row chunks (the library
+    # overlaps copy-in, compute and copy-out); `stream` completes after the
+    # last copy-out, so its events bracket all of it
     e2e_steps = max(1, min(args.steps, 3))
     ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(e2e_steps)]
-    for s in range(e2e_steps):
-        ee[s][0].record(stream)
-        for d, h in ((dq, hq), (dk, hk), (dv, hv)):
-            d.view(torch.int16).copy_(h, non_blocking=True)
-        layer_call(tri_layer)
-        ho.copy_(do.view(torch.int16), non_blocking=True)
-        ee[s][1].record(stream)
+    for s in range(e2e_steps + 1):  # the first call is a warm-up (copy streams created)
+        if s > 0:
+            ee[s - 1][0].record(stream)
+        tm.tm_trianglemix_attn_fwd_host(hq, hk, hv, ho, dq, dk, dv, do, wl.B, wl.Hq, wl.Hkv, wl.N,
+                                        wl.D, wl.scale, wl.S, W, wl.L, tri_layer, wl.tri_start, 0,
+                                        stream)
+        if s > 0:
+            ee[s - 1][1].record(stream)
     torch.cuda.synchronize()
     e2e_ms = sum(ee[s][0].elapsed_time(ee[s][1]) for s in range(e2e_steps)) / e2e_steps
 
@@ -416,7 +420,8 @@ def run_ours(args):
         "e2e": {"value": whole_job_tflops(ws, 1, tri_f, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": int((dq.numel() + dk.numel() + dv.numel()) * 2),
                 "d2h_bytes_per_step": int(do.numel() * 2),
-                "what": "pinned host q,k,v -> device, triangle layer, output -> pinned host"},
+                "what": "tm_trianglemix_attn_fwd_host: pinned host q,k,v -> device, triangle "
+                        "layer, output -> pinned host, streamed in 8192-row chunks"},
         "block_sparse": {
             "what": "tm_block_sparse_attn_fwd, seeded block index (local 8, sink 1, vertical 32, "
                     "slash 8 blocks per list), timed separately after the steps",

@@ -21,9 +21,12 @@
  *
  * Ownership and threading:
  *   - q, k, v, o are DEVICE pointers owned by the caller, 16-byte aligned;
- *     o must not overlap q, k or v. The library allocates no device memory
- *     in any call and keeps no per-call state; scratch for the split
- *     schedule is a caller-owned workspace (the *_ws calls).
+ *     o must not overlap q, k or v (tm_trianglemix_attn_fwd_host takes host
+ *     buffers besides them). The library allocates no device memory in any
+ *     call and keeps no per-call state; scratch for the split schedule is a
+ *     caller-owned workspace (the *_ws calls). The host-buffer call creates
+ *     two copy streams and a pool of events per device on first use and
+ *     keeps them for the life of the process.
  *   - `stream` is a cudaStream_t (CUstream) handle passed as void*; NULL is
  *     the legacy default stream. Work is enqueued asynchronously on it and
  *     the call returns without synchronising.
@@ -92,6 +95,40 @@ TM_API int tm_triangle_attn_fwd(const void* q, const void* k, const void* v, voi
 TM_API int tm_trianglemix_attn_fwd(const void* q, const void* k, const void* v, void* o, int B,
                                    int Hq, int Hkv, int N, int D, float scale, int S, int W,
                                    int L, int layer, int tri_start, void* stream);
+
+/*
+ * The same layer call on HOST buffers, streamed: q_host, k_host, v_host are
+ * read and o_host is written, in the [B, N, H, D] bf16 layout above.
+ * - Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister); a
+ *   pageable buffer still works, but its copies do not overlap.
+ * - q_dev, k_dev, v_dev, o_dev: caller-owned device buffers of the same sizes
+ *   and layout (16-byte aligned; o_dev overlapping none of the others), used
+ *   as staging. The library allocates no device memory.
+ * - The rows are taken in chunks of chunk_rows, a multiple of TM_BLOCK_M; 0
+ *   picks 8192. Chunks grow so that there are at most 64.
+ * - For chunk c, the library copies its q, k and v rows in on one internal
+ *   stream, then computes its queries on `stream` as soon as they and every
+ *   earlier chunk are resident, then copies its o rows out on a second
+ *   internal stream. In causal order a chunk's queries need no later key, so
+ *   copy-in, compute and copy-out of different chunks overlap.
+ * - The result is bit for bit that of tm_trianglemix_attn_fwd on the same
+ *   device buffers.
+ * - Ordering: the copies start after the work queued on `stream` before the
+ *   call, and `stream` completes only after the last copy-out. So the host
+ *   buffers may be reused once `stream` has been synchronised. The call
+ *   returns once all copies and kernels are queued.
+ * - Calls on one device are enqueued one at a time (the internal streams are
+ *   shared per device).
+ * - Errors: TM_ERR_INVALID_ARG for a NULL host pointer or a bad chunk_rows,
+ *   and otherwise as for tm_trianglemix_attn_fwd on the device buffers.
+ *   TM_ERR_CUDA if a copy or launch cannot be queued; work queued before the
+ *   failure still runs.
+ */
+TM_API int tm_trianglemix_attn_fwd_host(const void* q_host, const void* k_host,
+                                        const void* v_host, void* o_host, void* q_dev,
+                                        void* k_dev, void* v_dev, void* o_dev, int B, int Hq,
+                                        int Hkv, int N, int D, float scale, int S, int W, int L,
+                                        int layer, int tri_start, int chunk_rows, void* stream);
 
 /*
  * Triangle attention with a band per q head: head h keeps the sinks j < S_h
@@ -303,6 +340,16 @@ TM_API int tm_debug_mma_probe(const void* q, const void* k, const void* v, float
  */
 TM_API int tm_debug_schedule(int B, int Hq, int Hkv, int N, int causal, int S, int W, int L,
                              int num_ctas, int split, int* out, long long cap, long long* count);
+
+/*
+ * tm_debug_schedule for the work of the q-blocks [qb_lo, qb_hi) only (qb_hi
+ * -1: to the last q-block), the split that tm_trianglemix_attn_fwd_host runs
+ * for one row chunk; q-block numbers in the records are global. Requires
+ * 0 <= qb_lo < qb_hi <= ceil(N / TM_BLOCK_M). Host only.
+ */
+TM_API int tm_debug_schedule_window(int B, int Hq, int Hkv, int N, int causal, int S, int W,
+                                    int L, int num_ctas, int split, int qb_lo, int qb_hi,
+                                    int* out, long long cap, long long* count);
 
 /*
  * Failure-detection check (tests only): runs tm_triangle_attn_fwd with one

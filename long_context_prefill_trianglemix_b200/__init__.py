@@ -24,8 +24,10 @@ TM_BLOCK_M = TM_BLOCK_N = 128
 
 EXPORTED = (
     "tm_causal_attn_fwd", "tm_triangle_attn_fwd", "tm_trianglemix_attn_fwd",
+    "tm_trianglemix_attn_fwd_host",
     "tm_triangle_kept_pairs", "tm_kept_tiles", "tm_triangle_tile_list", "tm_tile_list",
-    "tm_debug_dump_tiles", "tm_debug_mma_probe", "tm_debug_schedule", "tm_get_device_status",
+    "tm_debug_dump_tiles", "tm_debug_mma_probe", "tm_debug_schedule", "tm_debug_schedule_window",
+    "tm_get_device_status",
     "tm_status_string", "tm_attn_workspace_size", "tm_causal_attn_fwd_ws", "tm_triangle_attn_fwd_ws",
     "tm_trianglemix_attn_fwd_ws", "tm_trianglemix_attn_fwd_noalloc", "tm_block_sparse_attn_fwd",
     "tm_trianglemix_sparse_attn_fwd", "tm_flashprefill_workspace_size",
@@ -58,6 +60,8 @@ def lib() -> ctypes.CDLL:
             "tm_triangle_attn_fwd": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci, ci, vp]),
             "tm_trianglemix_attn_fwd": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci, ci,
                                              ci, ci, vp]),
+            "tm_trianglemix_attn_fwd_host": (ci, [vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci,
+                                                  ci, cf, ci, ci, ci, ci, ci, ci, vp]),
             "tm_triangle_kept_pairs": (cll, [ci, ci, ci, ci]),
             "tm_kept_tiles": (cll, [ci, ci, ci, ci, ci]),
             "tm_triangle_tile_list": (ci, [ci, ci, ci, ci, ci, ci, vp, cll,
@@ -67,6 +71,8 @@ def lib() -> ctypes.CDLL:
             "tm_debug_mma_probe": (ci, [vp, vp, vp, vp, vp, ci, vp]),
             "tm_debug_schedule": (ci, [ci, ci, ci, ci, ci, ci, ci, ci, ci, ci, vp, cll,
                                        ctypes.POINTER(cll)]),
+            "tm_debug_schedule_window": (ci, [ci, ci, ci, ci, ci, ci, ci, ci, ci, ci, ci, ci, vp,
+                                              cll, ctypes.POINTER(cll)]),
             "tm_attn_workspace_size": (ci, [ci, ci, ci, ci, ci, ci, ci, ci, ci, ci,
                                             ctypes.POINTER(cll)]),
             "tm_causal_attn_fwd_ws": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp, cll, vp]),
@@ -141,6 +147,15 @@ def tm_trianglemix_attn_fwd(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L, layer,
     return _check("tm_trianglemix_attn_fwd", lib().tm_trianglemix_attn_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, Hkv, N, D, scale, S, W, L, layer, tri_start,
         _stream(stream)))
+
+
+def tm_trianglemix_attn_fwd_host(q_host, k_host, v_host, o_host, q_dev, k_dev, v_dev, o_dev, B,
+                                 Hq, Hkv, N, D, scale, S, W, L, layer, tri_start, chunk_rows=0,
+                                 stream=None):
+    return _check("tm_trianglemix_attn_fwd_host", lib().tm_trianglemix_attn_fwd_host(
+        _ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(o_host), _ptr(q_dev), _ptr(k_dev),
+        _ptr(v_dev), _ptr(o_dev), B, Hq, Hkv, N, D, scale, S, W, L, layer, tri_start,
+        int(chunk_rows), _stream(stream)))
 
 
 def tm_causal_attn_fwd_ws(q, k, v, o, B, Hq, Hkv, N, D, scale, workspace, workspace_bytes,
@@ -269,18 +284,19 @@ def tm_debug_mma_probe(q, k, v, s_out, o_out, D, stream=None):
 
 
 def tm_debug_schedule(B, Hq, Hkv, N, causal, S, W, L, num_ctas=148, split=False,
-                      mix_pairs=False) -> np.ndarray:
+                      mix_pairs=False, qb_lo=0, qb_hi=-1) -> np.ndarray:
     """Persistent work split as an int32 [n, 7] array:
-    (cta, item, q-block, head0, Q tiles, first tile, end tile)."""
+    (cta, item, q-block, head0, Q tiles, first tile, end tile); with a window,
+    the split of the q-blocks [qb_lo, qb_hi) only."""
     split = int(bool(split)) | (2 if mix_pairs else 0)
     cnt = ctypes.c_longlong(0)
-    _check("tm_debug_schedule", lib().tm_debug_schedule(B, Hq, Hkv, N, int(causal), S, W, L,
-                                                        num_ctas, int(split), None, 0,
-                                                        ctypes.byref(cnt)))
+    f = lib().tm_debug_schedule_window
+    _check("tm_debug_schedule_window", f(B, Hq, Hkv, N, int(causal), S, W, L, num_ctas,
+                                         int(split), qb_lo, qb_hi, None, 0, ctypes.byref(cnt)))
     out = np.zeros((max(cnt.value, 1), 7), np.int32)
-    _check("tm_debug_schedule", lib().tm_debug_schedule(B, Hq, Hkv, N, int(causal), S, W, L,
-                                                        num_ctas, int(split), out.ctypes.data,
-                                                        cnt.value, ctypes.byref(cnt)))
+    _check("tm_debug_schedule_window", f(B, Hq, Hkv, N, int(causal), S, W, L, num_ctas,
+                                         int(split), qb_lo, qb_hi, out.ctypes.data, cnt.value,
+                                         ctypes.byref(cnt)))
     return out[: cnt.value]
 
 

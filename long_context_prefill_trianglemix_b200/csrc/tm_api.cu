@@ -89,8 +89,11 @@ int scratch_address(void** out) {
 int run(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv, int N, int D,
         float scale, const trimix::Pattern& pat, void* ws, long long ws_bytes, void* stream,
         const int* bs_off = nullptr, const int* bs_idx = nullptr, long long bs_nnz = 0,
-        const int* hS = nullptr, const int* hW = nullptr, int inject_cta = -1) {
+        const int* hS = nullptr, const int* hW = nullptr, int inject_cta = -1, int qb_lo = 0,
+        int qb_hi = -1) {
   trimix::LaunchArgs a;
+  a.qb_lo = qb_lo;
+  a.qb_hi = qb_hi;
   a.hS = hS;
   a.hW = hW;
   a.inject_cta = inject_cta;
@@ -105,6 +108,59 @@ int run(const void* q, const void* k, const void* v, void* o, int B, int Hq, int
   a.ws_bytes = ws_bytes;
   a.stream = stream;
   return trimix::launch_attention(a);
+}
+
+// Copy streams and events of the host-buffer layer call, created once per
+// device and kept for the life of the process (no device memory). One lock
+// per device covers a call's enqueueing, so concurrent calls never interleave
+// their event records and waits.
+constexpr int kMaxStreamChunks = 64;
+constexpr int kDefaultChunkRows = 8192;
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, end = nullptr;
+  cudaEvent_t loaded[kMaxStreamChunks] = {}, computed[kMaxStreamChunks] = {};
+  std::mutex m;
+};
+constexpr int kMaxPipeDevices = 64;
+HostPipe g_pipes[kMaxPipeDevices];
+std::mutex g_pipes_mutex;
+
+int host_pipe(HostPipe** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return TM_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxPipeDevices) return TM_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_pipes_mutex);
+  HostPipe& hp = g_pipes[dev];
+  if (!hp.ready) {
+    const unsigned ef = cudaEventDisableTiming;
+    if (cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&hp.start, ef) != cudaSuccess ||
+        cudaEventCreateWithFlags(&hp.end, ef) != cudaSuccess)
+      return TM_ERR_CUDA;
+    for (int c = 0; c < kMaxStreamChunks; ++c)
+      if (cudaEventCreateWithFlags(&hp.loaded[c], ef) != cudaSuccess ||
+          cudaEventCreateWithFlags(&hp.computed[c], ef) != cudaSuccess)
+        return TM_ERR_CUDA;
+    hp.ready = true;
+  }
+  *out = &hp;
+  return TM_OK;
+}
+
+// Rows [r0, r1) of every batch of a [B, N, H, D] bf16 tensor, one copy per batch.
+int copy_rows(void* dst, const void* src, int B, int N, int H, int D, int r0, int r1,
+              cudaMemcpyKind kind, cudaStream_t st) {
+  const size_t row = static_cast<size_t>(H) * D * 2;
+  for (int b = 0; b < B; ++b) {
+    const size_t off = (static_cast<size_t>(b) * N + r0) * row;
+    if (cudaMemcpyAsync(static_cast<char*>(dst) + off, static_cast<const char*>(src) + off,
+                        static_cast<size_t>(r1 - r0) * row, kind, st) != cudaSuccess)
+      return TM_ERR_CUDA;
+  }
+  return TM_OK;
 }
 
 }  // namespace
@@ -160,6 +216,65 @@ TM_API int tm_trianglemix_attn_fwd(const void* q, const void* k, const void* v, 
                                    int layer, int tri_start, void* stream) {
   return tm_trianglemix_attn_fwd_ws(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L, layer,
                                     tri_start, nullptr, 0, stream);
+}
+
+TM_API int tm_trianglemix_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
+                                        void* o_host, void* q_dev, void* k_dev, void* v_dev,
+                                        void* o_dev, int B, int Hq, int Hkv, int N, int D,
+                                        float scale, int S, int W, int L, int layer, int tri_start,
+                                        int chunk_rows, void* stream) {
+  if (!q_host || !k_host || !v_host || !o_host) return TM_ERR_INVALID_ARG;
+  if (int rc = validate_common(q_dev, k_dev, v_dev, o_dev, B, Hq, Hkv, N, D, scale)) return rc;
+  if (layer < 0 || tri_start < 0) return TM_ERR_INVALID_ARG;
+  const bool causal = layer < tri_start;
+  if (!causal)
+    if (int rc = validate_pattern(S, W, L)) return rc;
+  if (chunk_rows < 0 || chunk_rows % TM_BLOCK_M != 0) return TM_ERR_INVALID_ARG;
+  if (chunk_rows == 0) chunk_rows = kDefaultChunkRows;
+  // at most kMaxStreamChunks chunks: larger chunks for longer sequences
+  const long long min_rows = (static_cast<long long>(N) + kMaxStreamChunks - 1) / kMaxStreamChunks;
+  if (chunk_rows < min_rows)
+    chunk_rows = static_cast<int>((min_rows + TM_BLOCK_M - 1) / TM_BLOCK_M * TM_BLOCK_M);
+  const int n_chunks = static_cast<int>((static_cast<long long>(N) + chunk_rows - 1) / chunk_rows);
+  const trimix::Pattern pat =
+      causal ? trimix::make_pattern(N, 1, 0, 1, 0) : trimix::make_pattern(N, 0, S, W, L);
+  HostPipe* hp = nullptr;
+  if (int rc = host_pipe(&hp)) return rc;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(hp->m);
+  // the copies start after the work already queued on the caller's stream
+  if (cudaEventRecord(hp->start, cs) != cudaSuccess ||
+      cudaStreamWaitEvent(hp->in, hp->start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(hp->out, hp->start, 0) != cudaSuccess)
+    return TM_ERR_CUDA;
+  for (int c = 0; c < n_chunks; ++c) {
+    const int r0 = c * chunk_rows;
+    const int r1 = std::min(N, r0 + chunk_rows);
+    // chunk c's queries need keys [0, r1) only: its own rows and the chunks before it
+    if (int rc = copy_rows(q_dev, q_host, B, N, Hq, D, r0, r1, cudaMemcpyHostToDevice, hp->in))
+      return rc;
+    if (int rc = copy_rows(k_dev, k_host, B, N, Hkv, D, r0, r1, cudaMemcpyHostToDevice, hp->in))
+      return rc;
+    if (int rc = copy_rows(v_dev, v_host, B, N, Hkv, D, r0, r1, cudaMemcpyHostToDevice, hp->in))
+      return rc;
+    if (cudaEventRecord(hp->loaded[c], hp->in) != cudaSuccess ||
+        cudaStreamWaitEvent(cs, hp->loaded[c], 0) != cudaSuccess)
+      return TM_ERR_CUDA;
+    if (int rc = run(q_dev, k_dev, v_dev, o_dev, B, Hq, Hkv, N, D, scale, pat, nullptr, 0, stream,
+                     nullptr, nullptr, 0, nullptr, nullptr, -1, r0 / TM_BLOCK_M,
+                     (r1 + TM_BLOCK_M - 1) / TM_BLOCK_M))
+      return rc;
+    if (cudaEventRecord(hp->computed[c], cs) != cudaSuccess ||
+        cudaStreamWaitEvent(hp->out, hp->computed[c], 0) != cudaSuccess)
+      return TM_ERR_CUDA;
+    if (int rc = copy_rows(o_host, o_dev, B, N, Hq, D, r0, r1, cudaMemcpyDeviceToHost, hp->out))
+      return rc;
+  }
+  // the caller's stream completes after the last copy-out
+  if (cudaEventRecord(hp->end, hp->out) != cudaSuccess ||
+      cudaStreamWaitEvent(cs, hp->end, 0) != cudaSuccess)
+    return TM_ERR_CUDA;
+  return TM_OK;
 }
 
 TM_API int tm_triangle_attn_fwd_heads(const void* q, const void* k, const void* v, void* o, int B,
@@ -382,17 +497,25 @@ TM_API int tm_debug_mma_probe(const void* q, const void* k, const void* v, float
   return trimix::launch_mma_probe(q, k, v, s_out, o_out, D, stream);
 }
 
-TM_API int tm_debug_schedule(int B, int Hq, int Hkv, int N, int causal, int S, int W, int L,
-                             int num_ctas, int split, int* out, long long cap, long long* count) {
+TM_API int tm_debug_schedule_window(int B, int Hq, int Hkv, int N, int causal, int S, int W,
+                                    int L, int num_ctas, int split, int qb_lo, int qb_hi, int* out,
+                                    long long cap, long long* count) {
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0 || num_ctas < 1 || cap < 0 || !count ||
       (cap > 0 && !out))
     return TM_ERR_INVALID_ARG;
   if (!causal && validate_pattern(S, W, L)) return TM_ERR_INVALID_ARG;
-  if (static_cast<long long>((N + TM_BLOCK_M - 1) / TM_BLOCK_M) * B * Hkv * ((Hq / Hkv + 1) / 2) >
-      (1LL << 31) - 1)
-    return TM_ERR_INVALID_ARG;
+  const long long nqb = (N + TM_BLOCK_M - 1) / TM_BLOCK_M;
+  if (nqb * B * Hkv * ((Hq / Hkv + 1) / 2) > (1LL << 31) - 1) return TM_ERR_INVALID_ARG;
+  if (qb_hi < 0) qb_hi = static_cast<int>(nqb);
+  if (qb_lo < 0 || qb_lo >= qb_hi || qb_hi > nqb) return TM_ERR_INVALID_ARG;
   return trimix::debug_schedule(B, Hq, Hkv, N, trimix::make_pattern(N, causal, S, W, L), num_ctas,
-                                split, out, cap, count);
+                                split, qb_lo, qb_hi, out, cap, count);
+}
+
+TM_API int tm_debug_schedule(int B, int Hq, int Hkv, int N, int causal, int S, int W, int L,
+                             int num_ctas, int split, int* out, long long cap, long long* count) {
+  return tm_debug_schedule_window(B, Hq, Hkv, N, causal, S, W, L, num_ctas, split, 0, -1, out, cap,
+                                  count);
 }
 
 TM_API int tm_debug_inject_stall(const void* q, const void* k, const void* v, void* o, int B,

@@ -136,7 +136,10 @@ struct Bars {
 static_assert(sizeof(Bars<8>) <= 256 && sizeof(Bars<4>) <= 256, "barrier block is 256 bytes");
 
 struct AttnParams {
-  int B, Hq, Hkv, N, G, npairs, nqb, units;
+  // nqb q-blocks of work, qb0 .. qb0 + nqb - 1 (a window of the nqb_all
+  // q-blocks of the sequence; the whole sequence unless the caller streams
+  // it in row chunks); q-block indices in items are global.
+  int B, Hq, Hkv, N, G, npairs, nqb, units, qb0, nqb_all;
   Pattern pat;
   float sl2;  // softmax scale * log2(e)
   // Items run q-block major (longest q-blocks first), the (batch, kv head,
@@ -177,7 +180,7 @@ struct AttnParams {
   int* ws_cnt;
   // Block-sparse launches (bs_off != nullptr): the tile list of item (b, kv
   // head g, q-block qb) is bs_idx[bs_off[r] .. bs_off[r + 1]), r = (b * Hkv +
-  // g) * nqb + qb, offsets clamped to [0, bs_nnz]; pat is the causal pattern.
+  // g) * nqb_all + qb, offsets clamped to [0, bs_nnz]; pat is the causal pattern.
   const int* bs_off;
   const int* bs_idx;
   int bs_nnz;
@@ -266,7 +269,7 @@ __host__ __device__ __forceinline__ Item decode_item(const AttnParams& p, int it
   Item it;
   const int qi = item / p.units;
   const int u = item - qi * p.units;
-  it.qb = p.nqb - 1 - qi;  // longest q-blocks first
+  it.qb = p.qb0 + p.nqb - 1 - qi;  // longest q-blocks first
   // unit digits, fastest first: pair, kv head, batch. The pairs of one kv head
   // and q-block are consecutive items, which the strided rounds hand to
   // neighbouring CTAs: they walk the same tile list in lockstep, so each K/V
@@ -325,9 +328,9 @@ __device__ __forceinline__ TileSrc tile_src(const AttnParams& p, const Item& it)
   TileSrc s;
   s.idx = nullptr;
   s.n = 0;
-  s.nkb = p.nqb;
+  s.nkb = p.nqb_all;
   if (p.bs_off) {
-    const long long r = (static_cast<long long>(it.b) * p.Hkv + it.g) * p.nqb + it.qb;
+    const long long r = (static_cast<long long>(it.b) * p.Hkv + it.g) * p.nqb_all + it.qb;
     const int o0 = imin(imax(__ldg(p.bs_off + r), 0), p.bs_nnz);
     const int o1 = imin(imax(__ldg(p.bs_off + r + 1), o0), p.bs_nnz);
     s.idx = p.bs_idx + o0;
@@ -410,7 +413,7 @@ struct WorkCursor {
       it.t1 = kAllTiles;
       it.split = -1;
       it.hunit = -1;
-      it.qb = p.nqb - 1 - qi;
+      it.qb = p.qb0 + p.nqb - 1 - qi;
       int ke = kvh + krot;
       if (ke >= p.Hkv) ke -= p.Hkv;
       it.g = ke;
@@ -1323,12 +1326,16 @@ int encode_bnhd(CUtensorMap* m, const void* base, int B, int N, int H, int D, in
 
 // Fills the geometry and the persistent work split of *p; returns the grid
 // size. split: heavy items may be cut into pieces (the caller has workspace).
+// The work is the q-blocks [qb0, qb0 + nqb_w) (nqb_w < 0: to the end).
 int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ctas, bool split,
-                   AttnParams* p, bool sparse = false, bool mix_pairs = false) {
+                   AttnParams* p, bool sparse = false, bool mix_pairs = false, int qb0 = 0,
+                   int nqb_w = -1) {
   p->B = B; p->Hq = Hq; p->Hkv = Hkv; p->N = N;
   p->G = Hq / Hkv;
   p->npairs = (p->G + 1) / 2;
-  p->nqb = (N + BM - 1) / BM;
+  p->nqb_all = (N + BM - 1) / BM;
+  p->qb0 = qb0;
+  p->nqb = nqb_w < 0 ? p->nqb_all - qb0 : nqb_w;
   p->units = B * Hkv * p->npairs;
   p->pat = pat;
   p->ws_rec = nullptr;
@@ -1349,7 +1356,7 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
   std::vector<long long> qcost(p->nqb);
   long long total = 0;
   for (int qb = 0; qb < p->nqb; ++qb) {
-    qcost[qb] = block_tiles(p->pat, qb, BM, BN).count() + kItemOverheadTiles;
+    qcost[qb] = block_tiles(p->pat, p->qb0 + qb, BM, BN).count() + kItemOverheadTiles;
     total += qcost[qb] * static_cast<long long>(B) * Hq;
   }
   const double target = static_cast<double>(total) / grid;
@@ -1379,10 +1386,11 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
   if (split && !sparse && n_hqb > 0) {
     const double heavy = static_cast<double>(qcost[p->nqb - 1] * item_q);
     ns = static_cast<int>(std::ceil(heavy / (kSplitShare * target)));
-    ns = std::min(ns, std::max(1, block_tiles(p->pat, p->nqb - 1, BM, BN).count() / kMinPieceTiles));
+    ns = std::min(ns, std::max(1, block_tiles(p->pat, p->qb0 + p->nqb - 1, BM, BN).count() /
+                                      kMinPieceTiles));
     ns = std::min(ns, kMaxSplit);
     while (n_sqb < n_hqb && qcost[p->nqb - 1 - n_sqb] * item_q > kSplitShare * target &&
-           block_tiles(p->pat, p->nqb - 1 - n_sqb, BM, BN).count() >= ns * kMinPieceTiles)
+           block_tiles(p->pat, p->qb0 + p->nqb - 1 - n_sqb, BM, BN).count() >= ns * kMinPieceTiles)
       ++n_sqb;
     ns = std::min(ns, std::max(1, static_cast<int>(
                               (8LL * grid - (n_hqb - n_sqb) * static_cast<long long>(p->units)) /
@@ -1470,7 +1478,7 @@ int launch_attention_d(const LaunchArgs& a, DeviceInfo* di) {
   const bool sparse = a.bs_off != nullptr;
   // per-head bands: pairs differ in cost, so every CTA cycles through the pairs
   const int grid = build_schedule(a.B, a.Hq, a.Hkv, a.N, a.pat, di->sms, a.ws != nullptr, &p,
-                                  sparse, a.hS != nullptr);
+                                  sparse, a.hS != nullptr, a.qb_lo, a.qb_hi - a.qb_lo);
   p.sl2 = a.scale * 1.4426950408889634f;
   p.inject_cta = a.inject_cta;
   if (a.hS) {  // per-head bands; a.pat already holds the maxima
@@ -1615,10 +1623,10 @@ int workspace_bytes(int B, int Hq, int Hkv, int N, int D, const Pattern& pat, in
 }
 
 int debug_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ctas, int split,
-                   int* out, long long cap, long long* count) {
+                   int qb_lo, int qb_hi, int* out, long long cap, long long* count) {
   AttnParams p;
-  const int grid =
-      build_schedule(B, Hq, Hkv, N, pat, max_ctas, (split & 1) != 0, &p, false, (split & 2) != 0);
+  const int grid = build_schedule(B, Hq, Hkv, N, pat, max_ctas, (split & 1) != 0, &p, false,
+                                  (split & 2) != 0, qb_lo, qb_hi - qb_lo);
   long long n = 0;
   for (int c = 0; c < grid; ++c) {
     WorkCursor cur;

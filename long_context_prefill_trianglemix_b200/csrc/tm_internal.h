@@ -28,6 +28,8 @@ struct LaunchArgs {
   const int* hW;
   int inject_cta;     // test hook: -1, or the CTA whose first Q is never delivered
   void* stream;
+  int qb_lo = 0;      // the q-blocks [qb_lo, qb_hi) of the sequence; qb_hi -1: to the end
+  int qb_hi = -1;
 };
 
 struct DiscArgs {
@@ -52,7 +54,7 @@ int read_and_clear_device_status(void* stream);
 int launch_discovery(const DiscArgs& a);
 long long discovery_workspace_bytes(int B, int Hq, int Hkv, int N, int D, int P);
 int debug_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ctas, int split,
-                   int* out, long long cap, long long* count);
+                   int qb_lo, int qb_hi, int* out, long long cap, long long* count);
 // Workspace bytes the split schedule needs on num_ctas CTAs (<= 0: the
 // current device's SM count); 0 if no item is split.
 int workspace_bytes(int B, int Hq, int Hkv, int N, int D, const Pattern& pat, int num_ctas,

@@ -206,3 +206,26 @@ def test_inject_stall_validates_before_launch():
     args = (FAKE, FAKE, FAKE, FAKE + 0x100000, 1, 4, 4, 64, 64, 0.1)
     assert tm.lib().tm_debug_inject_stall(*args, 4, 0, 2, None) == tm.TM_ERR_INVALID_ARG
     assert tm.lib().tm_debug_inject_stall(0, *args[1:], 4, 8, 2, None) == tm.TM_ERR_INVALID_ARG
+
+
+def test_host_streamed_call_validation():
+    """Every rejection happens before any CUDA call (none of these pointers is
+    ever dereferenced)."""
+    L = tm.lib()
+    H = 0x40000000  # stands for host buffers
+    dev = (FAKE, FAKE, FAKE, FAKE + 0x100000)
+    geo = (1, 4, 4, 64, 64, 0.1, 4, 8, 2)
+
+    def call(host=(H, H, H, H + 0x100000), devp=dev, geometry=geo, layer=1, tri_start=1, chunk=0):
+        return L.tm_trianglemix_attn_fwd_host(*host, *devp, *geometry, layer, tri_start, chunk,
+                                              None)
+    for i in range(4):  # a NULL host buffer
+        host = [H, H, H, H + 0x100000]
+        host[i] = 0
+        assert call(host=tuple(host)) == tm.TM_ERR_INVALID_ARG
+    assert call(devp=(0, FAKE, FAKE, FAKE + 0x100000)) == tm.TM_ERR_INVALID_ARG   # NULL device q
+    assert call(devp=(FAKE, FAKE, FAKE, FAKE + 0x100)) == tm.TM_ERR_INVALID_ARG   # o_dev aliases q
+    for chunk in (-128, 100, 129):                                                # not k * 128
+        assert call(chunk=chunk) == tm.TM_ERR_INVALID_ARG
+    assert call(layer=-1) == tm.TM_ERR_INVALID_ARG
+    assert call(geometry=(1, 4, 4, 64, 64, 0.1, 4, 0, 2)) == tm.TM_ERR_INVALID_ARG  # W = 0

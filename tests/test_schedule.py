@@ -208,3 +208,50 @@ def test_wide_windows_keep_last_rows_as_big_items(W):
         rec = tm.tm_debug_schedule(1, 32, 8, N, False, 64, W, L, 148, split=split)
         cost = cta_costs(rec, per_qb)
         assert cost.max() <= 1.02 * cost.mean(), (W, split, cost.max() / cost.mean())
+
+
+WINDOW_CASES = [  # B, Hq, Hkv, N, causal, S, W, L, chunk rows
+    (1, 32, 8, 32768, False, 64, 1024, 128, 4096),
+    (1, 32, 8, 32768, True, 0, 1, 0, 4096),
+    (1, 32, 8, 131072, False, 64, 2048, 256, 8192),
+    (2, 6, 2, 3000, False, 64, 300, 200, 512),
+    (1, 28, 4, 5000, True, 0, 1, 0, 1024),
+    (1, 14, 2, 777, False, 5, 200, 100, 128),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,causal,S,W,L,chunk", WINDOW_CASES)
+def test_row_chunk_windows_cover_each_item_once(B, Hq, Hkv, N, causal, S, W, L, chunk):
+    """The host-buffer call runs one launch per row chunk over the q-blocks of
+    that chunk; together the launches cover every (q-block, q head) once."""
+    nqb = (N + 127) // 128
+    seen = {}
+    for r0 in range(0, N, chunk):
+        lo, hi = r0 // 128, (min(N, r0 + chunk) + 127) // 128
+        rec = tm.tm_debug_schedule(B, Hq, Hkv, N, causal, S, W, L, 148, qb_lo=lo, qb_hi=hi)
+        assert len(rec) == (hi - lo) * B * Hkv * ((Hq // Hkv + 1) // 2)
+        assert rec[:, 2].min() >= lo and rec[:, 2].max() < hi
+        # the longest q-blocks of the chunk come first in each CTA (for causal
+        # and the triangle's last-L blocks: the highest q-blocks)
+        for c in np.unique(rec[:, 0]):
+            mine = rec[rec[:, 0] == c]
+            if causal:
+                assert mine[0, 2] == mine[:, 2].max()
+        for c, item, qb, h0, nv, t0, t1 in rec:
+            assert t0 == 0
+            for h in range(h0, h0 + nv):
+                assert (qb, h) not in seen
+                seen[(qb, h)] = 1
+    assert len(seen) == nqb * B * Hq
+
+
+def test_window_arguments_rejected():
+    import ctypes
+    cnt = ctypes.c_longlong(0)
+    L = tm.lib()
+    for lo, hi in ((-1, 4), (4, 4), (5, 4), (0, 9)):   # N = 1000: 8 q-blocks
+        assert L.tm_debug_schedule_window(1, 4, 2, 1000, 1, 0, 1, 0, 148, 0, lo, hi, None, 0,
+                                          ctypes.byref(cnt)) == tm.TM_ERR_INVALID_ARG
+    assert L.tm_debug_schedule_window(1, 4, 2, 1000, 1, 0, 1, 0, 148, 0, 3, -1, None, 0,
+                                      ctypes.byref(cnt)) == tm.TM_OK
+    assert cnt.value == 5 * 2 * 1
