@@ -134,16 +134,29 @@ int host_pipe(HostPipe** out) {
   std::lock_guard<std::mutex> lock(g_pipes_mutex);
   HostPipe& hp = g_pipes[dev];
   if (!hp.ready) {
+    // create everything, or release what was created and report the failure
     const unsigned ef = cudaEventDisableTiming;
-    if (cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking) != cudaSuccess ||
-        cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking) != cudaSuccess ||
-        cudaEventCreateWithFlags(&hp.start, ef) != cudaSuccess ||
-        cudaEventCreateWithFlags(&hp.end, ef) != cudaSuccess)
+    std::vector<cudaStream_t> streams;
+    std::vector<cudaEvent_t> events;
+    bool ok = true;
+    for (cudaStream_t* st : {&hp.in, &hp.out}) {
+      ok = ok && cudaStreamCreateWithFlags(st, cudaStreamNonBlocking) == cudaSuccess;
+      if (ok) streams.push_back(*st);
+    }
+    std::vector<cudaEvent_t*> slots = {&hp.start, &hp.end};
+    for (int c = 0; c < kMaxStreamChunks; ++c) {
+      slots.push_back(&hp.loaded[c]);
+      slots.push_back(&hp.computed[c]);
+    }
+    for (cudaEvent_t* e : slots) {
+      ok = ok && cudaEventCreateWithFlags(e, ef) == cudaSuccess;
+      if (ok) events.push_back(*e);
+    }
+    if (!ok) {
+      for (cudaEvent_t e : events) cudaEventDestroy(e);
+      for (cudaStream_t st : streams) cudaStreamDestroy(st);
       return TM_ERR_CUDA;
-    for (int c = 0; c < kMaxStreamChunks; ++c)
-      if (cudaEventCreateWithFlags(&hp.loaded[c], ef) != cudaSuccess ||
-          cudaEventCreateWithFlags(&hp.computed[c], ef) != cudaSuccess)
-        return TM_ERR_CUDA;
+    }
     hp.ready = true;
   }
   *out = &hp;
@@ -248,8 +261,8 @@ TM_API int tm_trianglemix_attn_fwd_host(const void* q_host, const void* k_host, 
       cudaStreamWaitEvent(hp->out, hp->start, 0) != cudaSuccess)
     return TM_ERR_CUDA;
   for (int c = 0; c < n_chunks; ++c) {
-    const int r0 = c * chunk_rows;
-    const int r1 = std::min(N, r0 + chunk_rows);
+    const int r0 = c * chunk_rows;  // < N
+    const int r1 = static_cast<int>(std::min<long long>(N, static_cast<long long>(r0) + chunk_rows));
     // chunk c's queries need keys [0, r1) only: its own rows and the chunks before it
     if (int rc = copy_rows(q_dev, q_host, B, N, Hq, D, r0, r1, cudaMemcpyHostToDevice, hp->in))
       return rc;
