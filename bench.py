@@ -22,6 +22,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -40,12 +41,21 @@ BM = BN = 128
 # triangle launch of the default workload (llama3-8b-128k, W=2048) from one ncu
 # capture of this bench command, keyed by the hash of the kernel sources it was
 # taken on; reported only while the sources still match (else null).
-TRAFFIC = {"6a46f4a3a726b6dd": 2.354e9 + 1.042e9}
+TRAFFIC = {"3462f43072dce1df": 2.354e9 + 1.042e9}
 
 # The C-ABI file holds argument checks, the layer dispatch and the host-buffer
 # copy pipeline: no device code and no work split, so it does not change what
-# a launch reads or writes. Every other source of the library is hashed.
+# a launch reads or writes. Every other source of the library is hashed, as
+# code (comments and layout do not count).
 _NOT_KERNEL = {"tm_api.cu"}
+
+
+def _code_only(text: str) -> str:
+    """Source text without // and /* */ comments, whitespace runs collapsed: a
+    change to comments or layout does not change the kernel."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
 
 
 def kernel_source_hash() -> str:
@@ -54,8 +64,8 @@ def kernel_source_hash() -> str:
                                            "*"))):
         if os.path.basename(p) in _NOT_KERNEL:
             continue
-        with open(p, "rb") as f:
-            h.update(f.read())
+        with open(p, encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -10,7 +10,7 @@
 //   warps 0-3  softmax warpgroup 0: rows of Q tile 0 (TMEM lanes 0..127)
 //   warps 4-7  softmax warpgroup 1: rows of Q tile 1
 //   warp  8    TMA producer (one elected thread): Q tiles, then K/V tiles
-//   warp  9    tcgen05 issuer (one thread) and TMEM owner
+//   warp  9    tcgen05 issuer (the warp in step, one elected lane issues) and TMEM owner
 //   warps 10-11 idle (they complete the third warpgroup for setmaxnreg)
 // The kernel is launched at 168 registers per thread (384 x 168 = 64512);
 // the third warpgroup drops to 88 and the softmax warpgroups rise to 208
@@ -607,7 +607,7 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, Bars<Cfg<D>::
   }
 }
 
-// The tcgen05 issuer: one thread issues every MMA of both Q tiles in the order
+// The tcgen05 issuer: one lane of warp 9 issues every MMA of both Q tiles in the order
 // O0+=P0.V_t, S0=Q0.K_{t+1}, O1+=P1.V_t, S1=Q1.K_{t+1}, and keeps that order
 // across item boundaries: after the last O0+=P0.V of an item it issues the
 // next item's first S0 (then, after O1+=P1.V, its S1), so one softmax
