@@ -3,7 +3,6 @@ the committed generator, and the float32 operation sequence of ex2_poly stays
 within the fitted relative-error bound of 2^x (far below bf16's 2^-9)."""
 import os
 import re
-import subprocess
 import sys
 
 import numpy as np

@@ -13,7 +13,7 @@ import pytest
 
 import long_context_prefill_trianglemix_b200 as tm
 from long_context_prefill_trianglemix_b200 import inputs as I
-from gpu_util import assert_close, from_dev, sample_rows
+from gpu_util import assert_close, sample_rows
 
 pytestmark = pytest.mark.gpu
 

@@ -7,7 +7,6 @@ from the index with numpy; the closed form for q = 0 (the mean of v over the
 kept keys); zeros for rows that keep nothing; and the synthetic index recipe's
 structure (sorted, causal, with its local band, sinks, verticals and slashes).
 """
-import math
 
 import numpy as np
 import pytest

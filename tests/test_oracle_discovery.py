@@ -7,7 +7,6 @@ import os
 from fractions import Fraction
 
 import numpy as np
-import pytest
 
 import oracle
 from long_context_prefill_trianglemix_b200 import inputs as I
