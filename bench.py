@@ -37,34 +37,44 @@ METRIC = "triangle-attn prefill TFLOP/s (kept tiles) at 128K; speedup vs own cau
 UNIT = "TFLOP/s"
 BM = BN = 128
 # Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the
-# triangle launch of the default workload (llama3-8b-128k, W=2048) from one ncu
-# capture of this bench command, keyed by the hash of the kernel sources it was
-# taken on; reported only while the sources still match (else null).
-TRAFFIC = {"3462f43072dce1df": 2.354e9 + 1.042e9}
-
-# The C-ABI file holds argument checks, the layer dispatch and the host-buffer
-# copy pipeline: no device code and no work split, so it does not change what
-# a launch reads or writes. Every other source of the library is hashed, as
-# code (comments and layout do not count).
-_NOT_KERNEL = {"tm_api.cu"}
+# triangle launch of the default workload (llama3-8b-128k, W=2048) from a
+# one-launch ncu capture, keyed by the hash of the build inputs it was taken
+# on; reported only while the sources still match (else null).
+TRAFFIC: dict = {}
 
 
 def _code_only(text: str) -> str:
-    """Source text without // and /* */ comments, whitespace runs collapsed: a
-    change to comments or layout does not change the kernel."""
+    """Source text without // and /* */ comments (and # comments in Python),
+    whitespace runs collapsed: a change to comments or layout does not change
+    the kernel."""
     text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
     text = re.sub(r"//[^\n]*", " ", text)
     return " ".join(text.split())
 
 
+def kernel_sources() -> list:
+    """The files kernel_source_hash covers."""
+    pkg = os.path.join(ROOT, "long_context_prefill_trianglemix_b200")
+    paths = [p for p in sorted(glob.glob(os.path.join(pkg, "csrc", "*")))
+             if not p.endswith(".py")]
+    paths += sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
+    paths.append(os.path.join(pkg, "build.py"))
+    return paths
+
+
 def kernel_source_hash() -> str:
+    """Hash of everything that decides what a launch does: every library
+    source (kernels, the C-ABI file with the layer dispatch and the schedule
+    choice), the public header (tile shape) and the build script (compile
+    flags), as code."""
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "long_context_prefill_trianglemix_b200", "csrc",
-                                           "*"))):
-        if os.path.basename(p) in _NOT_KERNEL:
-            continue
+    for p in kernel_sources():
         with open(p, encoding="utf-8") as f:
-            h.update(_code_only(f.read()).encode())
+            text = f.read()
+        if p.endswith(".py"):
+            text = re.sub(r"#[^\n]*", " ", text)
+        h.update(os.path.basename(p).encode())
+        h.update(_code_only(text).encode())
     return h.hexdigest()[:16]
 
 
@@ -154,9 +164,10 @@ def oracle_sample(wl, W, n_rows: int, seed: int, host, target_s: float = 0.0):
     import numpy as np
 
     import oracle
-    import long_context_prefill_trianglemix_b200 as tm
     q, k, v = host
-    tiles = tm.tm_tile_list(wl.N, False, wl.S, W, wl.L)
+    # the kept-tile credit comes from the oracle's own tile list, so this leg
+    # (and the reference arm) loads no part of the CUDA library
+    tiles = oracle.tile_list_rows(wl.N, False, wl.S, W, wl.L)
     per_qb = np.bincount(tiles[:, 0], minlength=(wl.N + BM - 1) // BM)
     cores = oracle.hardware_threads()
     while True:
@@ -231,6 +242,27 @@ def run_reference(args):
     return 0
 
 
+def algorithmic_bytes(wl) -> float:
+    """Minimum HBM bytes of one layer: q, k, v read once and o written once (bf16)."""
+    return 2.0 * wl.B * wl.N * wl.D * (2 * wl.Hq + 2 * wl.Hkv)
+
+
+def timed_calls(stream, calls, steps):
+    """Run each of `calls` once per step, timing every call with CUDA events on
+    `stream`; returns per-call lists of milliseconds."""
+    import torch
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in calls] for _ in range(steps)]
+    for s in range(steps):
+        for c, fn in enumerate(calls):
+            ev[s][c][0].record(stream)
+            fn()
+            ev[s][c][1].record(stream)
+    torch.cuda.synchronize()
+    return [[ev[s][c][0].elapsed_time(ev[s][c][1]) for s in range(steps)]
+            for c in range(len(calls))]
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -246,6 +278,12 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
     wl = I.WORKLOADS[args.workload]
     W = args.window or wl.W
+    if wl.layers > 2 and args.legs == "all":
+        rc = run_model(args, wl, W, ws, rank)
+        if ws > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return rc
     tri_layer, causal_layer = wl.tri_start, max(wl.tri_start - 1, 0)
     assert wl.tri_start >= 1
 
@@ -258,7 +296,6 @@ def run_ours(args):
     I.make_qkv(wl, tri_layer, out=host_np)
     dq, dk, dv = (t.cuda().view(torch.bfloat16) for t in (hq, hk, hv))
     do = torch.empty_like(dq)
-    ho = torch.empty(shp_q, dtype=torch.int16, pin_memory=True)
     stream = torch.cuda.current_stream()
 
     # workspace for the split schedule (allocated once, outside the timed region;
@@ -274,56 +311,133 @@ def run_ours(args):
                                       wl.S, W, wl.L, layer, wl.tri_start, wsbuf, ws_bytes, stream)
 
     tri_f, causal_f = tile_flop(wl, False, W), tile_flop(wl, True)
+    step = [lambda: layer_call(tri_layer)]
+    if args.legs != "triangle":
+        step.append(lambda: layer_call(causal_layer))
 
     for _ in range(args.warmup):
-        layer_call(tri_layer)
-        layer_call(causal_layer)
+        for fn in step:
+            fn()
     torch.cuda.synchronize()
     if tm.tm_get_device_status(stream) != tm.TM_OK:
         raise RuntimeError("device status not ok after warm-up")
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     sampler = ClockSampler(local)
     if ws > 1:
         dist.barrier()
     torch.cuda.synchronize()
     sampler.start()
     time.sleep(0.3)
+    launches0 = tm.tm_debug_launch_count()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(step) + 1)]
+          for _ in range(args.steps)]
     for s in range(args.steps):
         ev[s][0].record(stream)
-        layer_call(tri_layer)
-        ev[s][1].record(stream)
-        layer_call(causal_layer)
-        ev[s][2].record(stream)
+        for c, fn in enumerate(step):
+            fn()
+            ev[s][c + 1].record(stream)
     torch.cuda.synchronize()
+    launches = tm.tm_debug_launch_count() - launches0
     if ws > 1:
         dist.barrier()
     clocks = sampler.stop()
     status = tm.tm_get_device_status(stream)
     tri_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(args.steps)]
-    cau_ms = [ev[s][1].elapsed_time(ev[s][2]) for s in range(args.steps)]
-    total_ms = ev[0][0].elapsed_time(ev[-1][2])
+    cau_ms = ([ev[s][1].elapsed_time(ev[s][2]) for s in range(args.steps)]
+              if len(step) > 1 else [float("nan")])
+    total_ms = ev[0][0].elapsed_time(ev[-1][-1])
     tri_sum = sum(tri_ms)
 
-    # end to end through the host-buffer call: pinned host q, k, v in, the
-    # triangle layer, pinned host o out, streamed in row chunks (the library
-    # overlaps copy-in, compute and copy-out); `stream` completes after the
-    # last copy-out, so its events bracket all of it
-    e2e_steps = max(1, min(args.steps, 3))
-    ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(e2e_steps)]
-    for s in range(e2e_steps + 1):  # the first call is a warm-up (copy streams created)
-        if s > 0:
-            ee[s - 1][0].record(stream)
-        tm.tm_trianglemix_attn_fwd_host(hq, hk, hv, ho, dq, dk, dv, do, wl.B, wl.Hq, wl.Hkv, wl.N,
-                                        wl.D, wl.scale, wl.S, W, wl.L, tri_layer, wl.tri_start, 0,
-                                        stream)
-        if s > 0:
-            ee[s - 1][1].record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = sum(ee[s][0].elapsed_time(ee[s][1]) for s in range(e2e_steps)) / e2e_steps
+    extra = {}
+    e2e_ms = float("nan")
+    if args.legs == "all":
+        # end to end through the host-buffer call: pinned host q, k, v in, the
+        # triangle layer, pinned host o out, streamed in row chunks (the library
+        # overlaps copy-in, compute and copy-out); `stream` completes after the
+        # last copy-out, so its events bracket all of it
+        ho = torch.empty(shp_q, dtype=torch.int16, pin_memory=True)
 
-    # block-sparse shallow layer (next to the triangle path: a seeded vertical /
-    # slash / local block index, 128x128 blocks), timed on its own after the steps
+        def host_call():
+            tm.tm_trianglemix_attn_fwd_host(hq, hk, hv, ho, dq, dk, dv, do, wl.B, wl.Hq, wl.Hkv,
+                                            wl.N, wl.D, wl.scale, wl.S, W, wl.L, tri_layer,
+                                            wl.tri_start, 0, stream)
+
+        host_call()  # warm-up (the library creates its copy streams on first use)
+        e2e_steps = max(3, args.steps)
+        e2e_ms = sum(timed_calls(stream, [host_call], e2e_steps)[0]) / e2e_steps
+        extra = other_legs(args, wl, W, tm, dq, dk, dv, do, stream, sum(cau_ms) / len(cau_ms),
+                           tri_layer)
+
+    total_ms, tri_sum, e2e_ms = reduce_over_ranks([total_ms, tri_sum, e2e_ms], device="cuda")
+
+    peaks = load_peaks()
+    tri_avg = tri_sum / args.steps
+    achieved = tri_f / (tri_avg * 1e-3) / 1e12
+    value = whole_job_tflops(ws, args.steps, tri_f, tri_sum)
+    hbm_gbs = algorithmic_bytes(wl) / (tri_avg * 1e-3) / 1e9
+    causal_avg = sum(cau_ms) / len(cau_ms)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(wl, W, ws),
+        "split_workspace_bytes": ws_bytes,
+        "legs": args.legs,
+        "triangle_ms": tri_avg,
+        "triangle_ms_p10_p90": [float(np.percentile(tri_ms, 10)), float(np.percentile(tri_ms, 90))],
+        "causal_ms": causal_avg,
+        "causal_tflops": causal_f / (causal_avg * 1e-3) / 1e12,
+        "speedup_vs_causal": causal_avg / tri_avg,
+        "kept_tile_tflop": tri_f / 1e12,
+        "kept_pair_tflops": (tm.tm_triangle_kept_pairs(wl.N, wl.S, W, wl.L) * wl.B * wl.Hq * 4.0
+                             * wl.D) / (tri_avg * 1e-3) / 1e12,
+        "triangle_hbm": {"algorithmic_bytes": algorithmic_bytes(wl), "gbs": hbm_gbs,
+                         "frac_of_measured_hbm": hbm_gbs / peaks["hbm"],
+                         "what": "q, k, v read once and o written once, over the triangle "
+                                 "launch's time (the kernel is tensor-bound; this is context)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["sustained"],
+                     "unit": "TFLOP/s", "frac": achieved / peaks["sustained"],
+                     "peak_kind": f"bf16 dense, {peaks['source']} sustained (kernel runs inside "
+                                  "a long step after the causal layer)",
+                     "frac_of_burst": achieved / peaks["burst"],
+                     "traffic": TRAFFIC.get(kernel_source_hash()) if wl.name == "llama3-8b-128k"
+                     and W == 2048 else None},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "device_status": tm.status_string(status),
+    }
+    if args.legs == "all":
+        line["e2e"] = {
+            "value": whole_job_tflops(ws, 1, tri_f, e2e_ms), "unit": UNIT,
+            "h2d_bytes_per_step": int((dq.numel() + dk.numel() + dv.numel()) * 2),
+            "d2h_bytes_per_step": int(do.numel() * 2),
+            "what": "tm_trianglemix_attn_fwd_host: pinned host q,k,v -> device, triangle "
+                    "layer, output -> pinned host, streamed in 8192-row chunks; mean of %d calls"
+                    % max(3, args.steps)}
+        line.update(extra)
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        dt, equiv, cores, desc = oracle_sample(wl, W, args.cpu_rows, 7, host_np, target_s=10.0)
+        line["cpu_baseline"] = {"value": equiv / dt / 1e12, "unit": UNIT, "cores": cores,
+                                "kind": "oracle", "sample": desc, "seconds": dt}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0 if status == tm.TM_OK else 1
+
+
+def other_legs(args, wl, W, tm, dq, dk, dv, do, stream, causal_ms, tri_layer):
+    """The legs next to the headline step, each timed on its own after it: the
+    block-sparse shallow layer on a seeded index, per-head bands, and block
+    pattern discovery feeding block-sparse attention."""
+    import dataclasses
+
+    import numpy as np
+    import torch
+
+    # block-sparse shallow layer (a seeded vertical / slash / local block index,
+    # 128x128 blocks)
     bs_off, bs_idx = I.make_block_index(wl.B, wl.Hkv, wl.N, 0)
     d_off = torch.from_numpy(bs_off).cuda()
     d_idx = torch.from_numpy(bs_idx).cuda()
@@ -334,17 +448,11 @@ def run_ours(args):
 
     for _ in range(args.warmup):
         sparse_call()
-    bs_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    for s in range(args.steps):
-        bs_ev[s][0].record(stream)
-        sparse_call()
-        bs_ev[s][1].record(stream)
-    torch.cuda.synchronize()
-    bs_ms = sum(bs_ev[s][0].elapsed_time(bs_ev[s][1]) for s in range(args.steps))
+    bs_ms = float(np.mean(timed_calls(stream, [sparse_call], args.steps)[0]))
     bs_f = float(len(bs_idx)) * (wl.Hq // wl.Hkv) * 4.0 * BM * BN * wl.D
 
     # per-head bands (seeded windows 512..4096 and sinks {0, 64} per q head) on the
-    # same inputs, timed on its own; useful FLOPs count each head's own tiles
+    # same inputs; useful FLOPs count each head's own tiles
     hS, hW = I.head_bands(wl.Hq, 0)
     head_tiles = sum(tm.tm_kept_tiles(wl.N, False, int(hS[h]), int(hW[h]), wl.L)
                      for h in range(wl.Hq)) * wl.B
@@ -358,19 +466,12 @@ def run_ours(args):
 
     for _ in range(args.warmup):
         heads_call()
-    hb_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    for s in range(args.steps):
-        hb_ev[s][0].record(stream)
-        heads_call()
-        hb_ev[s][1].record(stream)
-    torch.cuda.synchronize()
-    hb_ms = sum(hb_ev[s][0].elapsed_time(hb_ev[s][1]) for s in range(args.steps))
+    hb_ms = float(np.mean(timed_calls(stream, [heads_call], args.steps)[0]))
 
     # block pattern discovery (probes per block, alpha) producing an index on the
-    # GPU, then block-sparse attention over it; both timed on their own. Seeded
-    # N(0,1) tensors have no attention structure to find, so this leg runs on the
-    # same shapes with the planted recipe (local and vertical structure).
-    import dataclasses
+    # GPU, then block-sparse attention over it. Seeded N(0,1) tensors have no
+    # attention structure to find, so this leg runs on the same shapes with the
+    # planted recipe (local and vertical structure).
     pwl = dataclasses.replace(wl, recipe="planted")
     pq, pk, _ = I.make_qkv(pwl, tri_layer)
     dq_p = torch.from_numpy(pq.view(np.int16)).cuda().view(torch.bfloat16)
@@ -395,93 +496,130 @@ def run_ours(args):
     for _ in range(args.warmup):
         discover_call()
         discovered_sparse_call()
-    dv_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    for s in range(args.steps):
-        dv_ev[s][0].record(stream)
-        discover_call()
-        dv_ev[s][1].record(stream)
-        discovered_sparse_call()
-        dv_ev[s][2].record(stream)
-    torch.cuda.synchronize()
-    disc_ms = sum(dv_ev[s][0].elapsed_time(dv_ev[s][1]) for s in range(args.steps))
-    dsa_ms = sum(dv_ev[s][1].elapsed_time(dv_ev[s][2]) for s in range(args.steps))
+    disc_t, dsa_t = timed_calls(stream, [discover_call, discovered_sparse_call], args.steps)
+    disc_ms, dsa_ms = float(np.mean(disc_t)), float(np.mean(dsa_t))
     f_nnz = int(f_off[-1].item())
-
-    total_ms, tri_sum, e2e_ms, bs_ms, disc_ms, dsa_ms, hb_ms = reduce_over_ranks(
-        [total_ms, tri_sum, e2e_ms, bs_ms, disc_ms, dsa_ms, hb_ms], device="cuda")
-
-    peaks = load_peaks()
-    tri_avg = tri_sum / args.steps
-    achieved = tri_f / (tri_avg * 1e-3) / 1e12
-    value = whole_job_tflops(ws, args.steps, tri_f, tri_sum)
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(workload_config(wl, W, ws), split_workspace_bytes=ws_bytes),
-        "triangle_ms": tri_avg,
-        "triangle_ms_p10_p90": [float(np.percentile(tri_ms, 10)), float(np.percentile(tri_ms, 90))],
-        "causal_ms": sum(cau_ms) / args.steps,
-        "causal_tflops": causal_f / (sum(cau_ms) / args.steps * 1e-3) / 1e12,
-        "speedup_vs_causal": (sum(cau_ms) / args.steps) / tri_avg,
-        "kept_tile_tflop": tri_f / 1e12,
-        "kept_pair_tflops": (tm.tm_triangle_kept_pairs(wl.N, wl.S, W, wl.L) * wl.B * wl.Hq * 4.0
-                             * wl.D) / (tri_avg * 1e-3) / 1e12,
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["sustained"],
-                     "unit": "TFLOP/s", "frac": achieved / peaks["sustained"],
-                     "peak_kind": f"bf16 dense, {peaks['source']} sustained (kernel runs inside "
-                                  "a long step after the causal layer)",
-                     "frac_of_burst": achieved / peaks["burst"],
-                     "traffic": TRAFFIC.get(kernel_source_hash())},
-        "e2e": {"value": whole_job_tflops(ws, 1, tri_f, e2e_ms), "unit": UNIT,
-                "h2d_bytes_per_step": int((dq.numel() + dk.numel() + dv.numel()) * 2),
-                "d2h_bytes_per_step": int(do.numel() * 2),
-                "what": "tm_trianglemix_attn_fwd_host: pinned host q,k,v -> device, triangle "
-                        "layer, output -> pinned host, streamed in 8192-row chunks"},
+    bs_ms, disc_ms, dsa_ms, hb_ms = reduce_over_ranks([bs_ms, disc_ms, dsa_ms, hb_ms],
+                                                      device="cuda")
+    return {
         "block_sparse": {
             "what": "tm_block_sparse_attn_fwd, seeded block index (local 8, sink 1, vertical 32, "
                     "slash 8 blocks per list), timed separately after the steps",
-            "ms": bs_ms / args.steps,
-            "tflops_kept_tiles": bs_f / (bs_ms / args.steps * 1e-3) / 1e12,
+            "ms": bs_ms,
+            "tflops_kept_tiles": bs_f / (bs_ms * 1e-3) / 1e12,
             "kept_tiles": int(len(bs_idx)) * (wl.Hq // wl.Hkv),
-            "density_vs_causal": len(bs_idx) / (wl.B * wl.Hkv * ((wl.N + BM - 1) // BM)
-                                                * ((wl.N + BM - 1) // BM + 1) / 2),
-            "speedup_vs_causal": (sum(cau_ms) / args.steps) / (bs_ms / args.steps),
+            "density_vs_causal": len(bs_idx) / (wl.B * wl.Hkv * nqb * (nqb + 1) / 2),
+            "speedup_vs_causal": causal_ms / bs_ms,
         },
         "head_bands": {
             "what": "tm_triangle_attn_fwd_heads, seeded per-head windows 512..4096 (log-uniform) "
                     "and sinks {0, 64}, L shared; heads paired in band order",
-            "ms": hb_ms / args.steps,
-            "tflops_own_tiles": head_tiles * 4.0 * BM * BN * wl.D / (hb_ms / args.steps * 1e-3)
-                                / 1e12,
+            "ms": hb_ms,
+            "tflops_own_tiles": head_tiles * 4.0 * BM * BN * wl.D / (hb_ms * 1e-3) / 1e12,
             "own_tiles": int(head_tiles),
-            "speedup_vs_causal": (sum(cau_ms) / args.steps) / (hb_ms / args.steps),
+            "speedup_vs_causal": causal_ms / hb_ms,
         },
         "discovery": {
             "what": "tm_flashprefill_block_index (pooled keys, %d probe rows per block and q "
                     "head, alpha %.2f) then tm_block_sparse_attn_fwd over the index it wrote; "
                     "q and k of the planted recipe (local and vertical structure)"
                     % (args.probes, args.alpha),
-            "speedup_vs_causal": (sum(cau_ms) / args.steps) / (dsa_ms / args.steps),
-            "discover_ms": disc_ms / args.steps,
-            "attention_ms": dsa_ms / args.steps,
+            "speedup_vs_causal": causal_ms / dsa_ms,
+            "discover_ms": disc_ms,
+            "attention_ms": dsa_ms,
             "density_vs_causal": f_nnz / (wl.B * wl.Hkv * nqb * (nqb + 1) / 2),
             "attention_tflops_kept_tiles": f_nnz * (wl.Hq // wl.Hkv) * 4.0 * BM * BN * wl.D
-                                           / (dsa_ms / args.steps * 1e-3) / 1e12,
+                                           / (dsa_ms * 1e-3) / 1e12,
         },
-        "gpu_launches": 2 * args.steps,
+    }
+
+
+def run_model(args, wl, W, ws, rank):
+    """All layers of a multi-layer workload, each with its own seeded inputs
+    (seed = layer), resident on the device. One step is one pass of the
+    TriangleMix schedule over every layer (causal below tri_start, triangle
+    from it); a second pass with every layer causal gives the dense total.
+    Totals are sums of the per-layer median times."""
+    import numpy as np
+    import torch
+
+    import long_context_prefill_trianglemix_b200 as tm
+
+    shp_q, shp_kv = (wl.B, wl.N, wl.Hq, wl.D), (wl.B, wl.N, wl.Hkv, wl.D)
+    hq = torch.empty(shp_q, dtype=torch.int16, pin_memory=True)
+    hk = torch.empty(shp_kv, dtype=torch.int16, pin_memory=True)
+    hv = torch.empty(shp_kv, dtype=torch.int16, pin_memory=True)
+    host_np = tuple(t.numpy().view(np.uint16) for t in (hq, hk, hv))
+    dev = []
+    for layer in range(wl.layers):
+        I.make_qkv(wl, layer, out=host_np)
+        dev.append(tuple(t.cuda().view(torch.bfloat16) for t in (hq, hk, hv)))
+    do = torch.empty_like(dev[0][0])
+    stream = torch.cuda.current_stream()
+    ws_bytes = 0
+    if args.split == "auto":
+        ws_bytes = max(tm.tm_attn_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.N, wl.D, causal, wl.S, W,
+                                                 wl.L) for causal in (False, True))
+    wsbuf = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device="cuda") if ws_bytes else None
+
+    def call(layer, tri_start):
+        q, k, v = dev[layer]
+        return lambda: tm.tm_trianglemix_attn_fwd_ws(q, k, v, do, wl.B, wl.Hq, wl.Hkv, wl.N, wl.D,
+                                                     wl.scale, wl.S, W, wl.L, layer, tri_start,
+                                                     wsbuf, ws_bytes, stream)
+
+    mix = [call(layer, wl.tri_start) for layer in range(wl.layers)]
+    dense = [call(layer, wl.layers) for layer in range(wl.layers)]  # every layer causal
+    for _ in range(args.warmup):
+        for fn in mix + dense:
+            fn()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    sampler.start()
+    time.sleep(0.3)
+    launches0 = tm.tm_debug_launch_count()
+    t_mix = timed_calls(stream, mix, args.steps)
+    t_dense = timed_calls(stream, dense, args.steps)
+    launches = tm.tm_debug_launch_count() - launches0
+    clocks = sampler.stop()
+    status = tm.tm_get_device_status(stream)
+    med_mix = [float(np.median(t)) for t in t_mix]
+    med_dense = [float(np.median(t)) for t in t_dense]
+    tri_layers = list(range(wl.tri_start, wl.layers))
+    tri_f = tile_flop(wl, False, W)
+    tri_ms = sum(med_mix[layer] for layer in tri_layers)
+    vals = reduce_over_ranks([tri_ms, sum(med_mix), sum(med_dense)], device="cuda")
+    tri_ms, mix_total, dense_total = vals
+    peaks = load_peaks()
+    achieved = tri_f * len(tri_layers) / (tri_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": ws * achieved, "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": mix_total,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": workload_config(wl, W, ws),
+        "model": {
+            "what": "every layer with its own seeded inputs (seed = layer); totals are sums of "
+                    "per-layer medians over the steps",
+            "layers": wl.layers, "tri_start": wl.tri_start,
+            "trianglemix_total_ms": mix_total,
+            "all_causal_total_ms": dense_total,
+            "attention_time_saved": 1.0 - mix_total / dense_total,
+            "speedup_vs_all_causal": dense_total / mix_total,
+            "causal_layers_ms": sum(med_mix[:wl.tri_start]),
+            "triangle_layers_ms": tri_ms,
+            "per_layer_ms": med_mix,
+            "per_layer_all_causal_ms": med_dense,
+        },
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["sustained"],
+                     "unit": "TFLOP/s", "frac": achieved / peaks["sustained"],
+                     "peak_kind": f"bf16 dense, {peaks['source']} sustained",
+                     "frac_of_burst": achieved / peaks["burst"], "traffic": None},
+        "gpu_launches": launches,
         "clocks": clocks,
         "device_status": tm.status_string(status),
     }
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        dt, equiv, cores, desc = oracle_sample(wl, W, args.cpu_rows, 7, host_np, target_s=10.0)
-        line["cpu_baseline"] = {"value": equiv / dt / 1e12, "unit": UNIT, "cores": cores,
-                                "kind": "oracle", "sample": desc, "seconds": dt}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if ws > 1:
-        dist.barrier()
-        dist.destroy_process_group()
     return 0 if status == tm.TM_OK else 1
 
 
@@ -500,6 +638,10 @@ def main():
     ap.add_argument("--alpha", type=float, default=0.3, help="discovery threshold factor")
     ap.add_argument("--split", choices=("auto", "off"), default="auto",
                     help="auto: give the launch the workspace that lets it cut long items")
+    ap.add_argument("--legs", choices=("all", "step", "triangle"), default="all",
+                    help="all: the step plus the e2e, block-sparse, per-head and discovery legs "
+                         "(multi-layer workloads: the whole model); step: the triangle + causal "
+                         "step only; triangle: the triangle layer only (for profiling)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps, always
     if args.impl == "reference":

@@ -260,17 +260,24 @@ TM_API int tm_trianglemix_attn_fwd_ws(const void* q, const void* k, const void* 
 
 /*
  * tm_trianglemix_attn_fwd with the split schedule, for callers that cannot
- * hand the library device memory: the paper has no counterpart. Instead of a
- * caller workspace it uses a fixed scratch array of TM_NOALLOC_SCRATCH_BYTES
- * (16 MiB) per device that the library's module holds; its address is looked
- * up once per device (cudaGetSymbolAddress). The call allocates and frees
- * nothing. A problem whose split schedule needs more scratch than that (as
- * reported by tm_attn_workspace_size on this device) is rejected with
- * TM_ERR_UNSUPPORTED before anything is enqueued; problems needing none run
- * without touching the scratch. Each call clears the arrival counters it
- * uses (an async memset on `stream`) before its kernel.
- * Calls that overlap in time on one device race on the scratch and give
- * undefined results: issue them on one stream, or order them otherwise.
+ * hand the library device memory: the paper has no counterpart. Callers that
+ * cannot allocate are, for instance, code running under a memory pool or a
+ * framework that owns every device byte, or code on a path where an
+ * allocation would synchronise the device. Instead of a caller workspace this
+ * call uses a fixed scratch array of TM_NOALLOC_SCRATCH_BYTES (16 MiB) that
+ * the library's module holds on every device that loads it, until the
+ * process exits. The call allocates and frees nothing. The array's address is
+ * looked up (cudaGetSymbolAddress) by the first call on each device context,
+ * and again after that context is recreated; make the first call outside any
+ * stream capture. A problem whose split needs more than the scratch (as
+ * tm_attn_workspace_size reports on this device) runs the unsplit schedule
+ * instead, which needs no scratch: the same attention, with the long items
+ * not cut (its bits may differ from a split run's in the last place); so does
+ * a problem with nothing to split. Each call that uses the scratch clears the
+ * arrival counters it needs (an async memset on `stream`) before its kernel;
+ * the rest of the array keeps the previous call's contents. Calls that
+ * overlap in time on one device race on the scratch and give undefined
+ * results: issue them on one stream, or order them otherwise.
  */
 #define TM_NOALLOC_SCRATCH_BYTES (16LL << 20)
 TM_API int tm_trianglemix_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o,
@@ -374,6 +381,16 @@ TM_API int tm_get_device_status(void* stream);
 
 /* Static string for a status code; never NULL. */
 TM_API const char* tm_status_string(int status);
+
+/*
+ * Number of kernels this library has launched in the calling process so far
+ * (every launch whose enqueue succeeded, on any device and stream; the
+ * host-buffer call's copies are not kernels and do not count). Read it
+ * before and after a region to count the library's launches inside it; the
+ * paper has no counterpart: it is measurement support. Host only, never
+ * fails.
+ */
+TM_API long long tm_debug_launch_count(void);
 
 #ifdef __cplusplus
 }

@@ -32,7 +32,7 @@ EXPORTED = (
     "tm_trianglemix_attn_fwd_ws", "tm_trianglemix_attn_fwd_noalloc", "tm_block_sparse_attn_fwd",
     "tm_trianglemix_sparse_attn_fwd", "tm_flashprefill_workspace_size",
     "tm_flashprefill_index_capacity", "tm_flashprefill_block_index", "tm_triangle_attn_fwd_heads",
-    "tm_debug_inject_stall",
+    "tm_debug_inject_stall", "tm_debug_launch_count",
 )
 
 
@@ -95,6 +95,7 @@ def lib() -> ctypes.CDLL:
             "tm_get_device_status": (ci, [vp]),
             "tm_debug_inject_stall": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci, ci, vp]),
             "tm_status_string": (ctypes.c_char_p, [ci]),
+            "tm_debug_launch_count": (cll, []),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -307,6 +308,10 @@ def tm_debug_inject_stall(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L, stream=N
 
 def tm_get_device_status(stream=None) -> int:
     return int(lib().tm_get_device_status(_stream(stream)))
+
+
+def tm_debug_launch_count() -> int:
+    return int(lib().tm_debug_launch_count())
 
 
 # ----------------------------------------------------------------------- torch conveniences

@@ -1,6 +1,7 @@
 // C ABI of the library (declared in include/tm.h): argument validation, the
 // layer schedule, host exports of the static tile list, and status handling.
 // All device work is delegated to tm_attn.cu.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -65,24 +66,63 @@ int validate_workspace(const void* q, const void* k, const void* v, const void* 
 
 // Scratch of tm_trianglemix_attn_fwd_noalloc: a fixed device array (one per
 // device, allocated with the module, never by a call) used as the split
-// workspace. Its address is looked up once per device.
+// workspace. Its address is looked up with cudaGetSymbolAddress once per
+// device context and cached under that context's unique id: a context that
+// is torn down and recreated (cudaDeviceReset) reloads the module, and the
+// next call looks the address up again instead of using a stale one.
 constexpr long long kScratchBytes = TM_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_split_scratch[kScratchBytes];
 
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+struct ScratchSlot {
+  unsigned long long ctx_id = 0;  // 0: not looked up yet
+  void* addr = nullptr;
+};
 std::mutex g_scratch_mutex;
-std::vector<void*> g_scratch_addr;  // per device; nullptr until looked up
+std::vector<ScratchSlot> g_scratch;  // per device ordinal
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+
+// Unique id of the calling thread's current context (0 if none is current).
+int current_context_id(unsigned long long* id) {
+  if (!g_ctx_get_current || !g_ctx_get_id) {
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+        q1 != cudaDriverEntryPointSuccess || !f1 ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+        q2 != cudaDriverEntryPointSuccess || !f2)
+      return TM_ERR_CUDA;
+    g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+    g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(f2);
+  }
+  CUcontext ctx = nullptr;
+  if (g_ctx_get_current(&ctx) != CUDA_SUCCESS) return TM_ERR_CUDA;
+  *id = 0;
+  if (ctx && g_ctx_get_id(ctx, id) != CUDA_SUCCESS) return TM_ERR_CUDA;
+  return TM_OK;
+}
 
 int scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return TM_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (static_cast<int>(g_scratch_addr.size()) <= dev) g_scratch_addr.resize(dev + 1, nullptr);
-  if (!g_scratch_addr[dev]) {
+  if (static_cast<int>(g_scratch.size()) <= dev) g_scratch.resize(dev + 1);
+  ScratchSlot& slot = g_scratch[dev];
+  unsigned long long id = 0;
+  if (int rc = current_context_id(&id)) return rc;
+  if (id == 0 || slot.ctx_id != id) {
+    // the lookup also makes the device's primary context current if none is
     void* a = nullptr;
     if (cudaGetSymbolAddress(&a, g_split_scratch) != cudaSuccess || !a) return TM_ERR_CUDA;
-    g_scratch_addr[dev] = a;
+    if (int rc = current_context_id(&id)) return rc;
+    slot.ctx_id = id;
+    slot.addr = a;
   }
-  *out = g_scratch_addr[dev];
+  *out = slot.addr;
   return TM_OK;
 }
 
@@ -430,12 +470,13 @@ TM_API int tm_trianglemix_attn_fwd_noalloc(const void* q, const void* k, const v
                                      : trimix::make_pattern(N, 0, S, W, L);
   long long need = 0;
   if (int rc = trimix::workspace_bytes(B, Hq, Hkv, N, D, pat, 0, &need)) return rc;
-  if (need > kScratchBytes) return TM_ERR_UNSUPPORTED;  // larger than the fixed scratch
+  // a split larger than the fixed scratch: run the unsplit schedule, which
+  // needs no scratch (the same attention; the long items are then not cut)
+  if (need == 0 || need > kScratchBytes)
+    return run(q, k, v, o, B, Hq, Hkv, N, D, scale, pat, nullptr, 0, stream);
   void* scratch = nullptr;
-  if (need > 0)
-    if (int rc = scratch_address(&scratch)) return rc;
-  return run(q, k, v, o, B, Hq, Hkv, N, D, scale, pat, scratch, need > 0 ? kScratchBytes : 0,
-             stream);
+  if (int rc = scratch_address(&scratch)) return rc;
+  return run(q, k, v, o, B, Hq, Hkv, N, D, scale, pat, scratch, kScratchBytes, stream);
 }
 
 TM_API long long tm_triangle_kept_pairs(int N, int S, int W, int L) {
@@ -541,6 +582,8 @@ TM_API int tm_debug_inject_stall(const void* q, const void* k, const void* v, vo
 }
 
 TM_API int tm_get_device_status(void* stream) { return trimix::read_and_clear_device_status(stream); }
+
+TM_API long long tm_debug_launch_count(void) { return trimix::kernel_launches(); }
 
 TM_API const char* tm_status_string(int status) {
   switch (status) {

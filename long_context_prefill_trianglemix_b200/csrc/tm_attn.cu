@@ -1264,6 +1264,15 @@ struct DeviceInfo {
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
+// Kernels this library has launched in the process (every launch site counts
+// itself once its launch returned without an error).
+std::atomic<long long> g_launches{0};
+
+int counted(int n) {
+  if (cudaGetLastError() != cudaSuccess) return TM_ERR_CUDA;
+  g_launches.fetch_add(n, std::memory_order_relaxed);
+  return TM_OK;
+}
 EncodeTiledFn g_encode = nullptr;
 DeviceInfo g_devices[kMaxDevices];  // fixed: pointers handed out stay valid
 
@@ -1513,7 +1522,7 @@ int launch_attention_d(const LaunchArgs& a, DeviceInfo* di) {
   }
   attn_kernel<D><<<grid, kThreads, Cfg<D>::kSmemBytes, static_cast<cudaStream_t>(a.stream)>>>(
       tq, tk, tv, to, p);
-  return cudaGetLastError() == cudaSuccess ? TM_OK : TM_ERR_CUDA;
+  return counted(1);
 }
 
 // [planes, rows, D] bf16 (D contiguous), 64-column x 128-row boxes, 128-byte swizzle.
@@ -1583,10 +1592,12 @@ int launch_discovery_d(const DiscArgs& a, DeviceInfo* di) {
   count_kernel<<<wblocks, 256, 0, st>>>(p);
   scan_kernel<<<1, 1024, 0, st>>>(p);
   write_index_kernel<<<wblocks, 256, 0, st>>>(p);
-  return cudaGetLastError() == cudaSuccess ? TM_OK : TM_ERR_CUDA;
+  return counted(5);
 }
 
 }  // namespace
+
+long long kernel_launches() { return g_launches.load(std::memory_order_relaxed); }
 
 long long discovery_workspace_bytes(int B, int Hq, int Hkv, int N, int D, int P) {
   return disc_layout(B, Hkv, N, D, (Hq / Hkv) * P).total;
@@ -1657,7 +1668,7 @@ int launch_dump_tiles(const Pattern& pat, int* out_dev, long long cap, void* str
   if (cap <= 0) return TM_OK;
   dump_tiles_kernel<<<(nqb + 127) / 128, 128, 0, static_cast<cudaStream_t>(stream)>>>(pat, nqb,
                                                                                       out_dev, cap);
-  return cudaGetLastError() == cudaSuccess ? TM_OK : TM_ERR_CUDA;
+  return counted(1);
 }
 
 template <int D>
@@ -1672,7 +1683,7 @@ static int launch_probe_d(const void* q, const void* k, const void* v, float* s_
     return TM_ERR_CUDA;
   mma_probe_kernel<D><<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, s_out,
                                                                           o_out);
-  return cudaGetLastError() == cudaSuccess ? TM_OK : TM_ERR_CUDA;
+  return counted(1);
 }
 
 int launch_mma_probe(const void* q, const void* k, const void* v, float* s_out, float* o_out,

@@ -51,6 +51,8 @@ int launch_dump_tiles(const Pattern& p, int* out_dev, long long cap, void* strea
 int launch_mma_probe(const void* q, const void* k, const void* v, float* s_out, float* o_out,
                      int D, void* stream);
 int read_and_clear_device_status(void* stream);
+// Kernels launched by the library so far in this process.
+long long kernel_launches();
 int launch_discovery(const DiscArgs& a);
 long long discovery_workspace_bytes(int B, int Hq, int Hkv, int N, int D, int P);
 int debug_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ctas, int split,

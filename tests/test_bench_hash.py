@@ -16,3 +16,9 @@ def test_code_changes_are_seen():
               "int f(int x) { return 2 * x; } int g;"):
         assert bench._code_only(a) != bench._code_only(b)
 
+
+
+def test_hash_covers_every_build_input():
+    names = {__import__("os").path.basename(p) for p in bench.kernel_sources()}
+    for must in ("tm_attn.cu", "tm_api.cu", "tm_sm100.cuh", "tm_tiles.cuh", "tm.h", "build.py"):
+        assert must in names, must

@@ -230,26 +230,46 @@ def llama128k():
     return wl, device_inputs(wl)
 
 
-def test_llama_128k_triangle_sampled_rows(llama128k):
+@pytest.fixture(scope="module")
+def llama128k_last_rows(llama128k):
+    """The oracle's output on all L = 256 last rows at 128K. Those rows keep every
+    causal key whatever S and W are (the pattern's last-Q-K region), so this one
+    fp64 computation is the expected value of the last rows of the triangle layer
+    at every window and of the causal layer."""
+    wl, (host, _) = llama128k
+    rows = list(range(wl.N - wl.L, wl.N))
+    return rows, oracle.attention(*host, wl.B, wl.Hq, wl.Hkv, wl.N, wl.D, wl.scale, True,
+                                  rows=rows)
+
+
+def check_last_rows(o_dev, last, what):
+    rows, want = last
+    return assert_close(from_dev(o_dev[:, rows[0]:rows[-1] + 1]), want, what + " (all last-L rows)")
+
+
+def test_llama_128k_triangle_sampled_rows(llama128k, llama128k_last_rows):
     wl, (host, (dq, dk, dv)) = llama128k
-    rows = sample_rows(wl.N, wl.L, 2, 64, 96, n_last=48)
+    rows = sample_rows(wl.N, wl.L, 2, 64, 96, n_last=0)
     o = run_dev(dq, dk, dv, wl, layer=1)
     check_rows(o, host, wl, False, rows, what="llama 128K triangle W=2048")
+    check_last_rows(o, llama128k_last_rows, "llama 128K triangle W=2048")
 
 
 @pytest.mark.parametrize("W", [512, 1024, 4096])
-def test_llama_128k_window_sweep_sampled_rows(llama128k, W):
+def test_llama_128k_window_sweep_sampled_rows(llama128k, llama128k_last_rows, W):
     wl, (host, (dq, dk, dv)) = llama128k
-    rows = sample_rows(wl.N, wl.L, 3, 32, 48, n_last=32)
+    rows = sample_rows(wl.N, wl.L, 3, 32, 48, n_last=0)
     o = run_dev(dq, dk, dv, wl, layer=1, W=W)
     check_rows(o, host, wl, False, rows, W=W, what=f"llama 128K triangle W={W}")
+    check_last_rows(o, llama128k_last_rows, f"llama 128K triangle W={W}")
 
 
-def test_llama_128k_causal_sampled_rows(llama128k):
+def test_llama_128k_causal_sampled_rows(llama128k, llama128k_last_rows):
     wl, (host, (dq, dk, dv)) = llama128k
-    rows = sample_rows(wl.N, wl.L, 4, 32, 32, n_last=16)
+    rows = sample_rows(wl.N, wl.L, 4, 32, 32, n_last=0)
     o = run_dev(dq, dk, dv, wl, layer=0)
     check_rows(o, host, wl, True, rows, what="llama 128K causal")
+    check_last_rows(o, llama128k_last_rows, "llama 128K causal")
 
 
 def test_llama_128k_zero_query_every_row(llama128k):
@@ -297,7 +317,7 @@ def test_qwen_128k_two_layers_sampled():
 def test_256k_context_sampled_rows_and_zero_query_every_row():
     """The longest context in the pages' experiments (the FlashPrefill summary
     reports 256K): N = 262144 with the Llama group shape on 8 q heads, the
-    split schedule on, sampled rows (all last-L rows) against the oracle and
+    split schedule on, sampled rows (all 256 last-L rows) against the oracle and
     the q = 0 closed form on every row."""
     import dataclasses
     import torch
@@ -311,7 +331,7 @@ def test_256k_context_sampled_rows_and_zero_query_every_row():
                                wl.W, wl.L, ws, n)
     torch.cuda.synchronize()
     assert tm.tm_get_device_status() == tm.TM_OK
-    rows = sample_rows(wl.N, wl.L, 13, 16, 48, n_last=64)
+    rows = sample_rows(wl.N, wl.L, 13, 16, 48)  # every one of the L last rows
     check_rows(o, (q, k, v), wl, False, rows, what="256K triangle")
     zq = torch.zeros_like(dq)
     tm.tm_triangle_attn_fwd_ws(zq, dk, dv, o, wl.B, wl.Hq, wl.Hkv, wl.N, wl.D, wl.scale, wl.S,

@@ -1,12 +1,17 @@
 """tm_trianglemix_attn_fwd_noalloc: the layer call with the split schedule on a
-fixed device scratch array instead of a caller workspace.
+fixed device scratch array instead of a caller workspace, for callers that
+cannot allocate device memory (a framework or pool that owns every device
+byte, or a path where an allocation would synchronise the device).
 
 On the GPU: two calls in a row give the same bits as the workspace entry
 point (the scratch's arrival counters are cleared by every call, so the
 second call does not see the first one's counts), for a triangle layer that
-is split and a causal layer that is not; a problem whose split needs more
-than the scratch is rejected before anything runs. Without a GPU: the symbol
-is exported and bad arguments are rejected before any CUDA call.
+is split and a causal layer; a triangle call and a causal call with
+different split layouts, enqueued back to back on one stream, each give the
+workspace entry point's bits; a problem whose split needs more than the
+scratch runs the unsplit schedule and gives the bits of the call without a
+workspace. Without a GPU: the symbol is exported and bad arguments are
+rejected before any CUDA call.
 """
 import math
 
@@ -59,11 +64,7 @@ def test_noalloc_matches_workspace_entry_two_calls_in_a_row(B, Hq, Hkv, N, D, S,
     compared = 0
     for layer in (1, 0):  # triangle (split), then causal (split or not, by shape)
         need = tm.tm_attn_workspace_size(B, Hq, Hkv, N, D, layer == 0, S, W, L)
-        if need > tm.TM_NOALLOC_SCRATCH_BYTES:  # refused before anything is enqueued
-            rc = tm.lib().tm_trianglemix_attn_fwd_noalloc(
-                q.data_ptr(), k.data_ptr(), v.data_ptr(), torch.empty_like(q).data_ptr(), B, Hq,
-                Hkv, N, D, scale, S, W, L, layer, 1, None)
-            assert rc == tm.TM_ERR_UNSUPPORTED
+        if need > tm.TM_NOALLOC_SCRATCH_BYTES:  # the unsplit fallback has its own test
             continue
         ws = torch.empty(max(need, 16), dtype=torch.uint8, device="cuda")
         ref = torch.empty_like(q)
@@ -84,19 +85,59 @@ def test_noalloc_matches_workspace_entry_two_calls_in_a_row(B, Hq, Hkv, N, D, S,
 
 
 @pytest.mark.gpu
-def test_noalloc_rejects_problems_larger_than_the_scratch():
+def test_noalloc_different_splits_back_to_back_on_one_stream():
+    """A triangle call and a causal call whose split schedules cut different
+    items into different numbers of pieces, enqueued alternately on one stream
+    with nothing in between: each call clears the counters its own layout
+    uses, so none sees the previous call's counts."""
     import torch
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
-    B, Hq, Hkv, N, D = 1, 2, 1, 32768, 128       # causal with two heads: many long items
-    need = tm.tm_attn_workspace_size(B, Hq, Hkv, N, D, True, 0, 1, 0)
-    assert need > tm.TM_NOALLOC_SCRATCH_BYTES
-    big_q = torch.zeros((B, N, Hq, D), dtype=torch.bfloat16, device="cuda")
-    big_kv = torch.zeros((B, N, Hkv, D), dtype=torch.bfloat16, device="cuda")
-    o = torch.empty_like(big_q)
-    rc = tm.lib().tm_trianglemix_attn_fwd_noalloc(big_q.data_ptr(), big_kv.data_ptr(),
-                                                  big_kv.data_ptr(), o.data_ptr(), B, Hq, Hkv,
-                                                  N, D, 0.1, 0, 1, 0, 0, 1, None)
-    assert rc == tm.TM_ERR_UNSUPPORTED
+    B, Hq, Hkv, N, D, S, W, L = 1, 2, 1, 8192, 64, 16, 256, 300
+    need = [tm.tm_attn_workspace_size(B, Hq, Hkv, N, D, layer == 0, S, W, L) for layer in (0, 1)]
+    assert 0 < need[1] < need[0] <= tm.TM_NOALLOC_SCRATCH_BYTES  # two different layouts
+    q, k, v = _inputs(B, Hq, Hkv, N, D, 43)
+    scale = 1.0 / math.sqrt(D)
+    refs = []
+    for layer in (0, 1):
+        ws = torch.empty(need[layer], dtype=torch.uint8, device="cuda")
+        ref = torch.empty_like(q)
+        tm.tm_trianglemix_attn_fwd_ws(q, k, v, ref, B, Hq, Hkv, N, D, scale, S, W, L, layer, 1,
+                                      ws, need[layer])
+        refs.append(ref)
+    torch.cuda.synchronize()
+    outs = []
+    for layer in (1, 0, 1, 0):
+        o = torch.full_like(q, float("nan"))
+        tm.tm_trianglemix_attn_fwd_noalloc(q, k, v, o, B, Hq, Hkv, N, D, scale, S, W, L, layer, 1)
+        outs.append((layer, o))
     torch.cuda.synchronize()
     assert tm.tm_get_device_status() == tm.TM_OK
+    for layer, o in outs:
+        assert torch.equal(o.view(torch.int16), refs[layer].view(torch.int16)), f"layer {layer}"
+
+
+@pytest.mark.gpu
+def test_noalloc_runs_unsplit_when_the_scratch_is_too_small():
+    """A causal layer with two heads at 32K cuts so many long items that its
+    split needs more than the scratch: the call runs the unsplit schedule,
+    whose bits are those of the call without a workspace."""
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    B, Hq, Hkv, N, D = 1, 2, 1, 32768, 128
+    need = tm.tm_attn_workspace_size(B, Hq, Hkv, N, D, True, 0, 1, 0)
+    assert need > tm.TM_NOALLOC_SCRATCH_BYTES
+    q, k, v = _inputs(B, Hq, Hkv, N, D, 47)
+    scale = 1.0 / math.sqrt(D)
+    ref = torch.empty_like(q)
+    tm.tm_trianglemix_attn_fwd(q, k, v, ref, B, Hq, Hkv, N, D, scale, 0, 1, 0, 0, 1)
+    outs = []
+    for _ in range(2):
+        o = torch.full_like(q, float("nan"))
+        tm.tm_trianglemix_attn_fwd_noalloc(q, k, v, o, B, Hq, Hkv, N, D, scale, 0, 1, 0, 0, 1)
+        outs.append(o)
+    torch.cuda.synchronize()
+    assert tm.tm_get_device_status() == tm.TM_OK
+    for o in outs:
+        assert torch.equal(o.view(torch.int16), ref.view(torch.int16))
