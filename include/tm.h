@@ -288,20 +288,30 @@ TM_API int tm_trianglemix_attn_fwd_noalloc(const void* q, const void* k, const v
 /*
  * Number of kept (i, j) pairs of one (batch, head) of the triangle pattern:
  * sum over rows of min(i+1, W) + max(0, min(S, i+1-W)) for i < N-L and i+1
- * otherwise. Host only. Returns -1 on a bad argument.
+ * otherwise. The kept set is the blog post's (TriangleMix blog post, section
+ * 介绍): the sink and local parts of the streaming region for most rows, and
+ * every causal key for the last L rows; the per-row closed form counts it with
+ * the window including the diagonal and the sinks and window as a union.
+ * Host only. Returns -1 on a bad argument.
  */
 TM_API long long tm_triangle_kept_pairs(int N, int S, int W, int L);
 
 /*
  * Number of TM_BLOCK_M x TM_BLOCK_N tiles the kernel visits for one
- * (batch, head): tiles holding at least one kept pair. causal != 0 counts
- * the causal pattern (S, W, L ignored). Host only. -1 on a bad argument.
+ * (batch, head): tiles holding at least one kept pair, the "kept tiles" whose
+ * FLOPs the throughput counts. Only these tiles are visited, by index, rather
+ * than branched over (FlashPrefill summary, section 2.3: physical jumps
+ * instead of logical skipping). causal != 0 counts the causal pattern (S, W,
+ * L ignored). Host only. -1 on a bad argument.
  */
 TM_API long long tm_kept_tiles(int N, int causal, int S, int W, int L);
 
 /*
  * Host export of the static tile list the kernels derive on the device, at
- * tile shape (BM, BN) (the kernels use TM_BLOCK_M x TM_BLOCK_N). One record is
+ * tile shape (BM, BN) (the kernels use TM_BLOCK_M x TM_BLOCK_N): the index by
+ * which the kernels jump from kept tile to kept tile (FlashPrefill summary,
+ * section 2.3), built from the triangle pattern's per-row kept intervals
+ * (TriangleMix blog post, section 介绍). One record is
  * three ints (qb, kb, full): q-block, k-block, and 1 if every pair of the
  * tile's existing rows and columns is kept (no mask needed), else 0. Records
  * are ordered by qb ascending, then kb ascending; tiles without a kept pair
@@ -315,10 +325,14 @@ TM_API int tm_tile_list(int N, int causal, int S, int W, int L, int BM, int BN, 
                         long long cap, long long* count);
 
 /*
- * Device dump of the same list, produced by the kernels' own device code at
- * TM_BLOCK_M x TM_BLOCK_N. out_dev: DEVICE buffer of 3*cap ints; *count
- * (host) receives the record total; records beyond cap are not written.
- * Asynchronous on `stream`.
+ * Device dump of the same list (FlashPrefill summary, section 2.3; TriangleMix
+ * blog post, section 介绍), produced by the kernels' own device code at
+ * TM_BLOCK_M x TM_BLOCK_N, so a test can compare what the device visits with
+ * the host list bit for bit. Beyond the plain dump of the triangle list it
+ * takes `causal` (the causal list, which the same device code produces) and
+ * returns the record total in *count (host), so the caller can size the
+ * buffer. out_dev: DEVICE buffer of 3*cap ints; records beyond cap are not
+ * written. Asynchronous on `stream`.
  */
 TM_API int tm_debug_dump_tiles(int N, int causal, int S, int W, int L, int* out_dev,
                                long long cap, long long* count, void* stream);

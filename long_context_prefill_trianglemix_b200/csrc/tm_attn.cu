@@ -72,9 +72,13 @@ constexpr int kWarpMma = 9;
 constexpr int kMaxCtas = 192;
 constexpr int kMaxBandHeads = 128;  // q heads of a per-head band launch
 constexpr uint32_t kTmemCols = 512;
-// Keep a stale running max until the true max exceeds it by 2^8: p stays <= 256
-// in fp32/bf16, and the O rescale (a TMEM round trip) becomes rare.
-constexpr float kRescaleThreshold = 8.0f;
+// Lazy running max (log2 domain): it moves only when a tile's max exceeds it
+// by more than kRescaleThreshold, and then to that max plus kRescaleMargin, so
+// the O rescale (a TMEM round trip on the softmax's critical path) stays rare
+// even when scores vary widely. Weights stay below 2^16 in fp32 and bf16, and
+// each new reference leaves them at most 2^-8 below their exact values' scale.
+constexpr float kRescaleThreshold = 16.0f;
+constexpr float kRescaleMargin = 8.0f;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 #ifndef TM_POLY_PAIRS
 #define TM_POLY_PAIRS 0
@@ -98,7 +102,7 @@ constexpr long long kSplitOverheadTiles = 1;
 // Where a wait gave up (recorded with the timeout, for diagnosis).
 enum WaitSite : int {
   kSiteQEmpty = 1, kSiteKvEmpty, kSiteQFull, kSiteKvFull, kSiteOEmpty, kSitePFull,
-  kSiteSFull, kSiteOFull, kSiteProbe, kSiteDisc
+  kSiteSFull, kSiteOFull, kSiteProbe, kSiteDisc, kSiteDescEmpty, kSiteDescFull
 };
 
 template <int D>
@@ -113,12 +117,19 @@ struct Cfg {
   static constexpr int kStageOff = kRingOff + kStages * kTileBytes;
   static constexpr int kStageSlotBytes = 32 * 128;
   static constexpr int kBarOff = kStageOff + 8 * kStageSlotBytes;
-  static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // barriers + alignment slack
+  static constexpr int kSmemBytes = kBarOff + 768 + 1024;  // barriers + alignment slack
   static constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128;
   static constexpr uint32_t kTmemO0 = 256, kTmemO1 = 256 + D;
   static constexpr uint32_t kIdescS = idesc_bf16_f32(BM, BN, 0, 0);  // Q, K both K-major
   static constexpr uint32_t kIdescO = idesc_bf16_f32(BM, D, 0, 1);   // V is MN-major
 };
+
+// What the producer tells the softmax warpgroups about each item, through a
+// ring of kDescRing slots in shared memory (qb < 0 ends the CTA's work).
+struct ItemDesc {
+  int b, g, qb, h0, h1, v1, t0, t1, split, hunit, pad0, pad1;
+};
+constexpr int kDescRing = 4;
 
 template <int NST>
 struct Bars {
@@ -132,8 +143,10 @@ struct Bars {
   // the CTA's work) and whether a second Q tile is present. Written before the
   // producer's arrival on q_full, read after the issuer's wait on it.
   int item_T, item_v1;
+  uint64_t desc_full[kDescRing], desc_empty[kDescRing];
+  ItemDesc desc[kDescRing];
 };
-static_assert(sizeof(Bars<8>) <= 256 && sizeof(Bars<4>) <= 256, "barrier block is 256 bytes");
+static_assert(sizeof(Bars<8>) <= 768 && sizeof(Bars<4>) <= 768, "barrier block is 768 bytes");
 
 struct AttnParams {
   // nqb q-blocks of work, qb0 .. qb0 + nqb - 1 (a window of the nqb_all
@@ -167,6 +180,17 @@ struct AttnParams {
   // kv_rot rotates the kv head the same way (per-head band launches, whose kv
   // heads differ in cost); it permutes whole groups, which stay adjacent too.
   int pair_rot, kv_rot;
+  // Chunked group order of the normal items (gchunk != 0; causal launches of
+  // even group sizes): the normal q-blocks are cut, from the longest, into
+  // chunks of qchunk q-blocks; chunk by chunk, every (batch, kv head) takes
+  // its turn with the chunk's q-blocks (longest first, pairs fastest). With
+  // qchunk = grid / npairs each turn is one strided round, so the CTAs running
+  // at the same time read the K/V of a single kv head, which stays in L2 for
+  // the whole round however far the CTAs drift apart along their tile lists;
+  // consecutive turns have the same cost profile, which the reversed odd
+  // rounds balance. The q-blocks left after the last full chunk (the
+  // shortest; their K/V fits in L2 for all heads) run q-block major.
+  int gchunk, qchunk;
   // Test hook (-1 in every product launch): the producer of this CTA delivers
   // no Q for its first item and leaves, so the issuer's bounded wait on q_full
   // runs out; the CTA records a timeout and every role exits cleanly.
@@ -342,119 +366,36 @@ __device__ __forceinline__ TileSrc tile_src(const AttnParams& p, const Item& it)
   return s;
 }
 
-// Walks one CTA's work (the same sequence as work_item) without an integer
-// division per item: a division costs a MUFU reciprocal, and MUFU is the unit
-// the softmax warps keep busy with exp2. Within each strided phase the item
-// index grows by a fixed stride, added digit by digit in the mixed radix
-// (pair, kv head, batch | q-block) of the item index.
-struct WorkCursor {
-  int k, n_work, nb, big_next, g, c;
-  int j, phase_end;                 // normal position; where the current stride ends
-  int pr, kvh, b, qi;               // digits of the next normal item
-  int d_pr, d_kvh, d_b, d_qi;       // digits of the current stride
-  int rot, d_rot;                   // qi * pair_rot and d_qi * pair_rot, mod npairs
-  int krot, d_krot;                 // qi * kv_rot and d_qi * kv_rot, mod Hkv
-  // main rounds alternate two strides (odd rounds run in reverse CTA order)
-  int e_pr, e_kvh, e_b, e_qi, e_rot, e_krot;  // digits of the other stride
-  int flip;                                  // 1: the strides alternate
-  __host__ __device__ __forceinline__ void set_item(const AttnParams& p, long long item) {
-    qi = static_cast<int>(item / p.units);
-    const int u = static_cast<int>(item - static_cast<long long>(qi) * p.units);
-    pr = u % p.npairs;
-    const int gb = u / p.npairs;
-    kvh = gb % p.Hkv;
-    b = gb / p.Hkv;
-    rot = static_cast<int>(static_cast<long long>(qi) * p.pair_rot % p.npairs);
-    krot = static_cast<int>(static_cast<long long>(qi) * p.kv_rot % p.Hkv);
-  }
-  __host__ __device__ __forceinline__ void set_stride(const AttnParams& p, int stride) {
-    d_qi = stride / p.units;
-    const int u = stride - d_qi * p.units;
-    d_pr = u % p.npairs;
-    const int gb = u / p.npairs;
-    d_kvh = gb % p.Hkv;
-    d_b = gb / p.Hkv;
-    d_rot = static_cast<int>(static_cast<long long>(d_qi) * p.pair_rot % p.npairs);
-    d_krot = static_cast<int>(static_cast<long long>(d_qi) * p.kv_rot % p.Hkv);
-  }
-  __host__ __device__ __forceinline__ void enter_phase(const AttnParams& p) {
-    set_item(p, p.n_hunits + normal_index(p, c, g, j));
-    const bool late = c >= p.n_a && j < p.n_skip;
-    phase_end = late ? p.n_skip : 0x7fffffff;
-    flip = late ? 0 : 1;
-    if (late) {
-      set_stride(p, g - p.n_a);
-      return;
-    }
-    // the main phase starts at round 0 (even): first 2g - 1 - 2c, then 2c + 1
-    set_stride(p, 2 * c + 1);
-    e_pr = d_pr; e_kvh = d_kvh; e_b = d_b; e_qi = d_qi; e_rot = d_rot; e_krot = d_krot;
-    set_stride(p, 2 * g - 1 - 2 * c);
-  }
-  __host__ __device__ __forceinline__ void init(const AttnParams& p, int cta, int grid) {
-    c = cta;
-    g = grid;
-    nb = big_count(p, c, g);
-    n_work = work_count(p, c, g);
-    k = 0;
-    big_next = c;
-    j = 0;
-    enter_phase(p);
-  }
-  __host__ __device__ __forceinline__ bool done() const { return k >= n_work; }
-  // Returns the next item of this CTA and advances.
-  __host__ __device__ __forceinline__ Item next(const AttnParams& p) {
-    Item it;
-    if (k < nb) {
-      it = decode_piece(p, big_next);
-      big_next += g;
-    } else {
-      it.t0 = 0;
-      it.t1 = kAllTiles;
-      it.split = -1;
-      it.hunit = -1;
-      it.qb = p.qb0 + p.nqb - 1 - qi;
-      int ke = kvh + krot;
-      if (ke >= p.Hkv) ke -= p.Hkv;
-      it.g = ke;
-      it.b = b;
-      int pe = pr + rot;
-      if (pe >= p.npairs) pe -= p.npairs;
-      pair_heads(p, ke, pe, it);
-      ++j;
-      if (j == phase_end) {
-        enter_phase(p);
-      } else {  // add the stride digit by digit
-        int carry = 0;
-        pr += d_pr;
-        if (pr >= p.npairs) { pr -= p.npairs; carry = 1; }
-        kvh += d_kvh + carry;
-        carry = 0;
-        if (kvh >= p.Hkv) { kvh -= p.Hkv; carry = 1; }
-        b += d_b + carry;
-        carry = 0;
-        if (b >= p.B) { b -= p.B; carry = 1; }
-        qi += d_qi + carry;
-        rot += d_rot + (carry ? p.pair_rot : 0);  // < 3 npairs
-        if (rot >= p.npairs) rot -= p.npairs;
-        if (rot >= p.npairs) rot -= p.npairs;
-        krot += d_krot + (carry ? p.kv_rot : 0);  // < 3 Hkv
-        if (krot >= p.Hkv) krot -= p.Hkv;
-        if (krot >= p.Hkv) krot -= p.Hkv;
-        if (flip) {  // swap to the other stride for the next step
-          int t0 = d_pr; d_pr = e_pr; e_pr = t0;
-          t0 = d_kvh; d_kvh = e_kvh; e_kvh = t0;
-          t0 = d_b; d_b = e_b; e_b = t0;
-          t0 = d_qi; d_qi = e_qi; e_qi = t0;
-          t0 = d_rot; d_rot = e_rot; e_rot = t0;
-          t0 = d_krot; d_krot = e_krot; e_krot = t0;
-        }
-      }
-    }
-    ++k;
-    return it;
-  }
-};
+// Normal item n (counted from 0 after the big items) in the launch's order.
+__host__ __device__ __forceinline__ Item normal_item(const AttnParams& p, long long n) {
+  const long long per_full = static_cast<long long>(p.qchunk) * p.units;
+  const long long n_chunked = (p.nqb - p.n_hqb) / p.qchunk * per_full;
+  // q-block major: every item without the chunked order, and the q-blocks
+  // after the last full chunk (the shortest ones) with it
+  if (!p.gchunk || n >= n_chunked) return decode_item(p, static_cast<int>(p.n_hunits + n));
+  const int k = static_cast<int>(n / per_full);      // chunk
+  const int rem = static_cast<int>(n - k * per_full);
+  const int per_gb = p.qchunk * p.npairs;
+  const int gb = rem / per_gb;
+  const int r2 = rem - gb * per_gb;
+  const int qi = p.n_hqb + k * p.qchunk + r2 / p.npairs;
+  Item it;
+  it.qb = p.qb0 + p.nqb - 1 - qi;
+  it.g = gb % p.Hkv;
+  it.b = gb / p.Hkv;
+  pair_heads(p, it.g, r2 % p.npairs, it);
+  it.t0 = 0;
+  it.t1 = kAllTiles;
+  it.split = -1;
+  it.hunit = -1;
+  return it;
+}
+
+// Item k of CTA c's work (big pieces first, then its normal items).
+__host__ __device__ __forceinline__ Item work_item_at(const AttnParams& p, int c, int g, int k) {
+  const int nb = big_count(p, c, g);
+  return k < nb ? decode_piece(p, c + k * g) : normal_item(p, normal_index(p, c, g, k - nb));
+}
 
 __device__ __forceinline__ void record_timeout(int site) {
   if (atomicCAS(&g_status, kDevOk, kDevTimeout) == kDevOk) g_status_where = site;
@@ -545,8 +486,18 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, Bars<Cfg<D>::
   const uint32_t ring = smem_addr(smem + Cfg<D>::kRingOff);
   uint32_t kv_cnt = 0, it_cnt = 0;
   bool ok = true;
-  WorkCursor cur;
-  cur.init(p, blockIdx.x, gridDim.x);
+  const int n_work = work_count(p, blockIdx.x, gridDim.x);
+  // Publishes item k's descriptor (or the end marker) for the softmax warpgroups.
+  auto publish = [&](int k, const Item& it, bool end) -> bool {
+    const int slot = k % kDescRing;
+    if (!wait_bar(&bars->desc_empty[slot], ((k / kDescRing) & 1) ^ 1, abort_flag, kSiteDescEmpty))
+      return false;
+    ItemDesc& d = bars->desc[slot];
+    d.b = it.b; d.g = it.g; d.qb = end ? -1 : it.qb; d.h0 = it.h0; d.h1 = it.h1; d.v1 = it.v1;
+    d.t0 = it.t0; d.t1 = it.t1; d.split = it.split; d.hunit = it.hunit;
+    mbar_arrive(&bars->desc_full[slot]);  // release: the descriptor is visible to the waiters
+    return true;
+  };
   // Per item: the first K/V tile goes into the ring before the wait for the Q
   // buffer (its ring slot frees about a tile earlier than the previous item's
   // last S releases Q, so it is in flight before Q), then Q, then the other
@@ -568,8 +519,9 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, Bars<Cfg<D>::
     }
     return true;
   };
-  while (ok && !cur.done()) {
-    const Item it = cur.next(p);
+  for (int k = 0; ok && k < n_work; ++k) {
+    const Item it = work_item_at(p, blockIdx.x, gridDim.x, k);
+    if (!(ok = publish(k, it, false))) break;
     const TileSrc bt = tile_src(p, it);
     const int t_end = imin(bt.count(), it.t1);
     if (t_end <= it.t0) continue;  // an empty block-sparse list: nothing to load
@@ -592,6 +544,7 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, Bars<Cfg<D>::
     ++it_cnt;
     for (int t = it.t0 + 1; ok && t < t_end; ++t) ok = load_kv(it, bt, t);
   }
+  if (ok) ok = publish(n_work, Item{}, true);  // the softmax warpgroups' end marker
   if (ok) {  // no more items: a descriptor of zero tiles, once Q is released
     if ((ok = wait_bar(&bars->q_empty, (it_cnt & 1u) ^ 1u, abort_flag, kSiteQEmpty))) {
       bars->item_T = 0;
@@ -891,10 +844,20 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
   const uint32_t tO = tmem_base + lane_addr + (wg ? Cfg<D>::kTmemO1 : Cfg<D>::kTmemO0);
   const float sl2 = p.sl2;
   uint32_t s_cnt = 0, o_cnt = 0;
-  WorkCursor cur;
-  cur.init(p, blockIdx.x, gridDim.x);
-  while (!cur.done()) {
-    const Item it = cur.next(p);
+  for (int k = 0;; ++k) {
+    // the producer's descriptor of this CTA's next item (qb < 0: no more)
+    const int ds = k % kDescRing;
+    const bool okd = wait_bar(&bars->desc_full[ds], (k / kDescRing) & 1, abort_flag, kSiteDescFull);
+    if (!__all_sync(0xffffffffu, okd)) return;
+    Item it;
+    {
+      const ItemDesc& d = bars->desc[ds];
+      it.b = d.b; it.g = d.g; it.qb = d.qb; it.h0 = d.h0; it.h1 = d.h1; it.v1 = d.v1;
+      it.t0 = d.t0; it.t1 = d.t1; it.split = d.split; it.hunit = d.hunit;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars->desc_empty[ds]);
+    if (it.qb < 0) break;
     if (wg == 1 && !it.v1) continue;
     const TileSrc bt = tile_src(p, it);
     const int T = imin(bt.count(), it.t1) - it.t0;
@@ -953,8 +916,8 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
       const bool bump = m_new > m_run + kRescaleThreshold;
       float alpha = 1.f;
       if (bump) {
-        alpha = ex2(m_run - m_new);
-        m_run = m_new;
+        alpha = ex2(m_run - (m_new + kRescaleMargin));
+        m_run = m_new + kRescaleMargin;
       }
       const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
       // O must be rescaled before the first half of this tile's P.V is issued
@@ -971,7 +934,10 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
       }
       // p = 2^(s * scale * log2 e - m): packed fp32x2 FMA, then exp2; l sums the
       // same bf16-rounded weights that P.V uses (exact widening adds), so O / l is
-      // a properly normalised average of v (a single dominant key returns v exactly).
+      // a properly normalised average of v (a single dominant key returns v exactly;
+      // summing the unrounded fp32 weights instead saves an instruction per pair
+      // but leaves O off by up to 2^-9 of |v| for peaked rows, which outlier-channel
+      // inputs push past the tolerance once the bf16 output rounding is added).
       // P is published in two halves (keys 0-63, 64-127): the MMA issuer starts
       // the first half of P.V while the second half is still being exponentiated.
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -1080,6 +1046,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->o_empty[w], 128);
     }
     mbar_init(&bars->mma_done, 1);
+    for (int r = 0; r < kDescRing; ++r) {
+      mbar_init(&bars->desc_full[r], 1);
+      mbar_init(&bars->desc_empty[r], 8);  // one arrival per softmax warp
+    }
     bars->abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -1356,6 +1326,8 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
   p->bs_idx = nullptr;
   p->bs_nnz = 0;
   p->ph = 0;
+  p->gchunk = 0;
+  p->qchunk = 1;
   // Persistent grid. Item cost = (visited tiles + fixed per-item overhead,
   // about the pipeline fill/drain and epilogue) x Q tiles of the item; it is
   // used to find the heavy q-blocks, how finely to cut them, and how many
@@ -1421,8 +1393,12 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
     }
     return 0;
   };
+  if (p->pat.causal && !sparse && !mix_pairs && p->G % 2 == 0 && n_hqb == 0 && grid >= p->npairs) {
+    p->gchunk = 1;
+    p->qchunk = grid / p->npairs;
+  }
   const int d_qi = grid / p->units;
-  if ((p->G % 2 == 1 || mix_pairs) && p->npairs > 1)
+  if (!p->gchunk && (p->G % 2 == 1 || mix_pairs) && p->npairs > 1)
     p->pair_rot = coprime_rotation((grid % p->units) % p->npairs, d_qi, p->npairs);
   if (mix_pairs && p->Hkv > 1)
     p->kv_rot = coprime_rotation((grid % p->units) / p->npairs % p->Hkv, d_qi, p->Hkv);
@@ -1640,18 +1616,10 @@ int debug_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
                                   (split & 2) != 0, qb_lo, qb_hi - qb_lo);
   long long n = 0;
   for (int c = 0; c < grid; ++c) {
-    WorkCursor cur;
-    cur.init(p, c, grid);
-    if (cur.n_work != work_count(p, c, grid)) return TM_ERR_INVALID_ARG;
-    for (int k = 0; !cur.done(); ++k, ++n) {
-      const Item it = cur.next(p);  // what the kernel's roles see
+    const int n_work = work_count(p, c, grid);
+    for (int k = 0; k < n_work; ++k, ++n) {
+      const Item it = work_item_at(p, c, grid, k);  // what the producer publishes
       const int item = work_item(p, c, grid, k);
-      const Item ref = item < p.n_big ? decode_piece(p, item)
-                                      : decode_item(p, item - p.n_big + p.n_hunits);
-      if (it.qb != ref.qb || it.b != ref.b || it.g != ref.g || it.h0 != ref.h0 || it.h1 != ref.h1 ||
-          it.v1 != ref.v1 ||
-          it.t0 != ref.t0 || it.t1 != ref.t1 || it.split != ref.split || it.hunit != ref.hunit)
-        return TM_ERR_INVALID_ARG;  // the cursor and the direct decode disagree
       if (n >= cap) continue;
       const int T = block_tiles(p.pat, it.qb, BM, BN).count();
       int* r = out + 7 * n;

@@ -68,15 +68,23 @@ def test_triangle_split_is_balanced(N, S, W, L):
 @pytest.mark.parametrize("N,causal,W,L", [(32768, False, 1024, 128), (131072, False, 2048, 256),
                                           (131072, True, 1, 0), (32768, True, 1, 0)])
 def test_concurrent_items_share_kv_tiles(N, causal, W, L):
-    # Items are dealt in strided rounds: each round of 148 consecutive items (what
-    # the CTAs run at about the same time) spans a narrow band of q-blocks of every
-    # kv head.
+    # Items are dealt in strided rounds: the 148 consecutive items of a round are
+    # what the CTAs run at about the same time. In a triangle launch a round spans
+    # a narrow band of q-blocks of every kv head. In a causal launch (chunked
+    # group order) a round holds the q-blocks of one chunk of a single kv head,
+    # so the K/V it reads is one head's (64 MB at 128K) and stays in L2; the
+    # shortest q-blocks after the last full chunk run like the triangle's.
     rec = tm.tm_debug_schedule(1, 32, 8, N, causal, 64, W, L, 148)
     order = np.argsort(rec[:, 1])
-    items, qbs = rec[order, 1], rec[order, 2]
+    items, qbs, kvh = rec[order, 1], rec[order, 2], rec[order, 3] // 4
     for r0 in range(0, len(items) - 148, 148):
         band = qbs[r0:r0 + 148]
-        assert band.max() - band.min() <= 10, (r0, band.min(), band.max())
+        full_chunks = (N // 128) // 74 * 74 * 16   # items of the full chunks
+        if causal and r0 + 148 <= full_chunks:
+            assert len(set(kvh[r0:r0 + 148].tolist())) == 1, r0
+            assert band.max() - band.min() < 74, (r0, band.min(), band.max())
+        else:
+            assert band.max() - band.min() <= 10, (r0, band.min(), band.max())
     # each CTA's items increase; odd rounds run in reverse CTA order, so a CTA's
     # strides alternate between 2g - 1 - 2c and 2c + 1 (they sum to two rounds)
     for c in range(148):
@@ -85,6 +93,16 @@ def test_concurrent_items_share_kv_tiles(N, causal, W, L):
         assert (d > 0).all(), (c, it[:6])
         main = d[-6:][d[-6:] < 2 * 148]   # normal items (big pieces have their own ids)
         assert set(main.tolist()) <= {2 * 148 - 1 - 2 * c, 2 * c + 1}, (c, main[:6])
+
+
+@pytest.mark.parametrize("N,Hq,Hkv", [(131072, 32, 8), (65536, 32, 8), (32768, 32, 8),
+                                      (131072, 4, 1), (65536, 8, 2)])
+def test_causal_chunked_group_order_is_balanced(N, Hq, Hkv):
+    rec = tm.tm_debug_schedule(1, Hq, Hkv, N, True, 0, 1, 0, 148)
+    cost = np.zeros(148)
+    for c, item, qb, h0, nv, t0, t1 in rec:
+        cost[c] += (qb + 1 + 3) * nv
+    assert cost.max() / cost.mean() <= 1.01, cost.max() / cost.mean()
 
 
 SPLIT_CASES = [(1, 4, 1, 131072, False, 64, 2048, 256), (1, 4, 1, 131072, False, 64, 512, 256),
