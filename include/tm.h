@@ -350,14 +350,16 @@ TM_API int tm_debug_mma_probe(const void* q, const void* k, const void* v, float
  * Host export of the persistent work split the kernels use on a grid of
  * num_ctas CTAs (the SM count on a B200). split: bit 0 gives the split
  * schedule of the *_ws calls (else the one of the calls without workspace),
- * bit 1 the pair rotation of per-head band launches. One record of
- * seven ints per work item, (cta, item, q-block, first q head
- * (batch * Hq + head), number of Q tiles 1 or 2, first tile, end tile), in the
- * order each CTA processes them; the tiles are positions [first, end) in the
- * q-block's tile list (the whole list unless the item is a piece). An item
- * covers one q-block of one or two q heads that share a kv head. out: HOST
- * buffer of 7*cap ints (NULL when cap = 0); *count receives the total. Host
- * only.
+ * bit 1 the item layout of per-head band launches (q-block pairs of one head
+ * for non-causal patterns, and the rotations). One record of seven ints per
+ * work item, (cta, item, q-block, first q head (batch * Hq + head), Q tiles,
+ * first tile, end tile), in the order each CTA processes them; the tiles are
+ * positions [first, end) in the item's tile list (the whole list unless the
+ * item is a piece). An item covers one q-block of one or two q heads that
+ * share a kv head; with q-block pairs (Q tiles has bit 8 set, 256 + 1 or 256 +
+ * 2), one or two consecutive q-blocks of one head, whose tile list is the
+ * union of theirs. out: HOST buffer of 7*cap ints (NULL when cap = 0); *count
+ * receives the total. Host only.
  */
 TM_API int tm_debug_schedule(int B, int Hq, int Hkv, int N, int causal, int S, int W, int L,
                              int num_ctas, int split, int* out, long long cap, long long* count);
@@ -371,6 +373,16 @@ TM_API int tm_debug_schedule(int B, int Hq, int Hkv, int N, int causal, int S, i
 TM_API int tm_debug_schedule_window(int B, int Hq, int Hkv, int N, int causal, int S, int W,
                                     int L, int num_ctas, int split, int qb_lo, int qb_hi,
                                     int* out, long long cap, long long* count);
+
+/*
+ * tm_debug_schedule of a per-head band launch (tm_triangle_attn_fwd_heads)
+ * with these bands: S_heads, W_heads are HOST arrays of Hq ints, as there.
+ * The bands decide which CTAs sit out rounds for holding an extra heavy item.
+ * Host only.
+ */
+TM_API int tm_debug_schedule_heads(int B, int Hq, int Hkv, int N, const int* S_heads,
+                                   const int* W_heads, int L, int num_ctas, int split, int* out,
+                                   long long cap, long long* count);
 
 /*
  * Failure-detection check (tests only): runs tm_triangle_attn_fwd with one

@@ -32,7 +32,7 @@ EXPORTED = (
     "tm_trianglemix_attn_fwd_ws", "tm_trianglemix_attn_fwd_noalloc", "tm_block_sparse_attn_fwd",
     "tm_trianglemix_sparse_attn_fwd", "tm_flashprefill_workspace_size",
     "tm_flashprefill_index_capacity", "tm_flashprefill_block_index", "tm_triangle_attn_fwd_heads",
-    "tm_debug_inject_stall", "tm_debug_launch_count",
+    "tm_debug_inject_stall", "tm_debug_launch_count", "tm_debug_schedule_heads",
 )
 
 
@@ -96,6 +96,8 @@ def lib() -> ctypes.CDLL:
             "tm_debug_inject_stall": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci, ci, vp]),
             "tm_status_string": (ctypes.c_char_p, [ci]),
             "tm_debug_launch_count": (cll, []),
+            "tm_debug_schedule_heads": (ci, [ci, ci, ci, ci, vp, vp, ci, ci, ci, vp, cll,
+                                             ctypes.POINTER(cll)]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -298,6 +300,22 @@ def tm_debug_schedule(B, Hq, Hkv, N, causal, S, W, L, num_ctas=148, split=False,
     _check("tm_debug_schedule_window", f(B, Hq, Hkv, N, int(causal), S, W, L, num_ctas,
                                          int(split), qb_lo, qb_hi, out.ctypes.data, cnt.value,
                                          ctypes.byref(cnt)))
+    return out[: cnt.value]
+
+
+def tm_debug_schedule_heads(B, Hq, Hkv, N, S_heads, W_heads, L, num_ctas=148,
+                            split=False) -> np.ndarray:
+    """tm_debug_schedule of a per-head band launch with these bands (records as there)."""
+    hs = np.ascontiguousarray(S_heads, dtype=np.int32)
+    hw = np.ascontiguousarray(W_heads, dtype=np.int32)
+    cnt = ctypes.c_longlong(0)
+    f = lib().tm_debug_schedule_heads
+    _check("tm_debug_schedule_heads", f(B, Hq, Hkv, N, hs.ctypes.data, hw.ctypes.data, L, num_ctas,
+                                        int(bool(split)), None, 0, ctypes.byref(cnt)))
+    out = np.zeros((max(cnt.value, 1), 7), np.int32)
+    _check("tm_debug_schedule_heads", f(B, Hq, Hkv, N, hs.ctypes.data, hw.ctypes.data, L, num_ctas,
+                                        int(bool(split)), out.ctypes.data, cnt.value,
+                                        ctypes.byref(cnt)))
     return out[: cnt.value]
 
 

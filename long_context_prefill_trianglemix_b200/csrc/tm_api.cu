@@ -566,6 +566,25 @@ TM_API int tm_debug_schedule_window(int B, int Hq, int Hkv, int N, int causal, i
                                 split, qb_lo, qb_hi, out, cap, count);
 }
 
+TM_API int tm_debug_schedule_heads(int B, int Hq, int Hkv, int N, const int* S_heads,
+                                   const int* W_heads, int L, int num_ctas, int split, int* out,
+                                   long long cap, long long* count) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0 || Hq > 128 || num_ctas < 1 ||
+      cap < 0 || !count || (cap > 0 && !out) || !S_heads || !W_heads || L < 0)
+    return TM_ERR_INVALID_ARG;
+  int S_max = 0, W_max = 1;
+  for (int h = 0; h < Hq; ++h) {
+    if (S_heads[h] < 0 || W_heads[h] < 1) return TM_ERR_INVALID_ARG;
+    S_max = std::max(S_max, S_heads[h]);
+    W_max = std::max(W_max, W_heads[h]);
+  }
+  const long long nqb = (N + TM_BLOCK_M - 1) / TM_BLOCK_M;
+  if (nqb * B * Hq > (1LL << 31) - 1) return TM_ERR_INVALID_ARG;
+  return trimix::debug_schedule(B, Hq, Hkv, N, trimix::make_pattern(N, 0, S_max, W_max, L),
+                                num_ctas, (split & 1) | 2, 0, static_cast<int>(nqb), out, cap,
+                                count, S_heads, W_heads);
+}
+
 TM_API int tm_debug_schedule(int B, int Hq, int Hkv, int N, int causal, int S, int W, int L,
                              int num_ctas, int split, int* out, long long cap, long long* count) {
   return tm_debug_schedule_window(B, Hq, Hkv, N, causal, S, W, L, num_ctas, split, 0, -1, out, cap,

@@ -215,6 +215,14 @@ struct AttnParams {
   // item visits the union of its two heads' tile lists, which is the closed
   // form at (max S, max W) since both kept sets are [0, S) U [i - W + 1, i].
   int ph;
+  // Q-block pairs (qpair != 0: per-head band launches): the two Q tiles of an
+  // item are consecutive q-blocks qb, qb + 1 of one q head instead of two
+  // heads of a group, so the union of their tile lists wastes about one tile
+  // per Q tile (heads of one group can have very different bands). The
+  // schedule's q-block x is then the pair of q-blocks 2x - qdelta, 2x + 1 -
+  // qdelta (qdelta puts the first full-causal q-block of the last-L rows at
+  // the start of a pair); a pair cut by the sequence's ends holds one Q tile.
+  int qpair, qdelta;
   int hS[kMaxBandHeads], hW[kMaxBandHeads];
   unsigned char hperm[kMaxBandHeads];
 };
@@ -282,11 +290,29 @@ __host__ __device__ __forceinline__ Pattern head_pattern(const AttnParams& p, in
 }
 __host__ __device__ __forceinline__ Pattern item_pattern(const AttnParams& p, const Item& it) {
   Pattern q = p.pat;
-  if (p.ph) {
+  if (p.ph && !p.qpair) {
     q.S = imax(p.hS[it.h0], p.hS[it.h1]);
     q.W = imax(p.hW[it.h0], p.hW[it.h1]);
+  } else if (p.ph) {
+    q.S = p.hS[it.h0];
+    q.W = p.hW[it.h0];
   }
   return q;
+}
+
+// Rows of schedule q-block x: [r0, r1] (two q-blocks with q-block pairs), and
+// the tile list of an item (the union of its Q tiles' lists).
+__host__ __device__ __forceinline__ BlockTiles sched_tiles(const AttnParams& p, const Pattern& pat,
+                                                           int x) {
+  if (!p.qpair) return block_tiles(pat, x, BM, BN);
+  const int qa = 2 * x - p.qdelta;
+  const int r0 = imax(qa, 0) * BM;
+  return block_tiles_rows(pat, r0, imin(p.N, (qa + 2) * BM) - 1, BN);
+}
+__host__ __device__ __forceinline__ BlockTiles item_tiles(const AttnParams& p, const Item& it) {
+  if (!p.qpair) return block_tiles(item_pattern(p, it), it.qb, BM, BN);
+  return block_tiles_rows(item_pattern(p, it), it.qb * BM,
+                          imin(p.N, (it.qb + 1 + it.v1) * BM) - 1, BN);
 }
 
 __host__ __device__ __forceinline__ Item decode_item(const AttnParams& p, int item) {
@@ -303,7 +329,14 @@ __host__ __device__ __forceinline__ Item decode_item(const AttnParams& p, int it
   const int gb = u / p.npairs;
   it.g = (gb % p.Hkv + static_cast<int>(static_cast<long long>(qi) * p.kv_rot % p.Hkv)) % p.Hkv;
   it.b = gb / p.Hkv;
-  pair_heads(p, it.g, pr, it);
+  if (p.qpair) {  // q-block pair (qa, qa + 1) of head pr of kv group g
+    const int qa = 2 * it.qb - p.qdelta;
+    it.qb = imax(qa, 0);
+    it.v1 = (qa >= 0 && qa + 1 < p.nqb_all) ? 1 : 0;
+    it.h0 = it.h1 = it.g * p.G + pr;
+  } else {
+    pair_heads(p, it.g, pr, it);
+  }
   it.t0 = 0;
   it.t1 = kAllTiles;
   it.split = -1;
@@ -323,7 +356,7 @@ __host__ __device__ __forceinline__ Item decode_piece(const AttnParams& p, int b
   const int u = rem - s * p.units;
   Item it = decode_item(p, qi * p.units + u);
   if (p.nsplit > 1) {
-    const int T = block_tiles(item_pattern(p, it), it.qb, BM, BN).count();
+    const int T = item_tiles(p, it).count();
     it.t0 = static_cast<int>(static_cast<long long>(T) * s / p.nsplit);
     it.t1 = static_cast<int>(static_cast<long long>(T) * (s + 1) / p.nsplit);
     it.split = s;
@@ -361,7 +394,7 @@ __device__ __forceinline__ TileSrc tile_src(const AttnParams& p, const Item& it)
     s.n = o1 - o0;
     s.bt.n_a = s.bt.b_lo = s.bt.n_b = 0;
   } else {
-    s.bt = block_tiles(item_pattern(p, it), it.qb, BM, BN);
+    s.bt = item_tiles(p, it);
   }
   return s;
 }
@@ -539,7 +572,7 @@ __device__ __forceinline__ void producer_role(const AttnParams& p, Bars<Cfg<D>::
       tma_load_4d(q0 + pn * Cfg<D>::kPanelBytes, tq, &bars->q_full, pn * 64, it.h0, it.qb * BM, it.b);
       if (it.v1)
         tma_load_4d(q0 + Cfg<D>::kTileBytes + pn * Cfg<D>::kPanelBytes, tq, &bars->q_full, pn * 64,
-                    it.h1, it.qb * BM, it.b);
+                    it.h1, (it.qb + p.qpair) * BM, it.b);
     }
     ++it_cnt;
     for (int t = it.t0 + 1; ok && t < t_end; ++t) ok = load_kv(it, bt, t);
@@ -863,7 +896,8 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
     const int T = imin(bt.count(), it.t1) - it.t0;
     const int head = wg ? it.h1 : it.h0;
     const Pattern pat = head_pattern(p, head);  // this Q tile's own mask
-    const int i = it.qb * BM + r;  // query row of this thread
+    const int my_qb = it.qb + (p.qpair ? wg : 0);  // this Q tile's q-block
+    const int i = my_qb * BM + r;  // query row of this thread
     // kept keys of row i: [0, sink_hi) U [band_lo, hi)
     const int hi = imin(i, pat.N - 1) + 1;
     const bool full_row = pat.causal || i >= pat.N - pat.L;
@@ -873,7 +907,7 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
     for (int t = 0; t < T; ++t) {
       const int kb = bt.kb(it.t0 + t);  // read before the wait, which hides its latency
       const bool bad = kb < 0;          // a clamped negative index entry: fully masked
-      const bool need_mask = bad || tile_needs_mask(pat, it.qb, kb, BM, BN) != 0;
+      const bool need_mask = bad || tile_needs_mask(pat, my_qb, kb, BM, BN) != 0;
       bool ok = wait_bar(&bars->s_full[wg], s_cnt & 1u, abort_flag, kSiteSFull);
       ++s_cnt;
       if (!__all_sync(0xffffffffu, ok)) return;
@@ -1007,8 +1041,8 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, Bars<Cfg<D>::k
       }
       fence_proxy_async_smem();  // make the generic-proxy writes visible to the TMA engine
       __syncwarp();
-      if (lane == 0 && it.qb * BM + wq * 32 < p.N) {  // a slot wholly past N stores nothing
-        tma_store_4d(to, slot, 64 * h, head, it.qb * BM + wq * 32, it.b);
+      if (lane == 0 && my_qb * BM + wq * 32 < p.N) {  // a slot wholly past N stores nothing
+        tma_store_4d(to, slot, 64 * h, head, my_qb * BM + wq * 32, it.b);
         bulk_commit_group();
       }
     }
@@ -1308,7 +1342,7 @@ int encode_bnhd(CUtensorMap* m, const void* base, int B, int N, int H, int D, in
 // The work is the q-blocks [qb0, qb0 + nqb_w) (nqb_w < 0: to the end).
 int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ctas, bool split,
                    AttnParams* p, bool sparse = false, bool mix_pairs = false, int qb0 = 0,
-                   int nqb_w = -1) {
+                   int nqb_w = -1, const int* hS = nullptr, const int* hW = nullptr) {
   p->B = B; p->Hq = Hq; p->Hkv = Hkv; p->N = N;
   p->G = Hq / Hkv;
   p->npairs = (p->G + 1) / 2;
@@ -1328,6 +1362,18 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
   p->ph = 0;
   p->gchunk = 0;
   p->qchunk = 1;
+  p->qpair = 0;
+  p->qdelta = 0;
+  if (mix_pairs && !sparse && !pat.causal && qb0 == 0 && (nqb_w < 0 || nqb_w == p->nqb_all)) {
+    // per-head band launches: items are q-block pairs of one head; the first
+    // q-block whose list is full causal (it holds last-L rows) starts a pair
+    p->qpair = 1;
+    const int kf = p->pat.L > 0 ? (N - p->pat.L) / BM : p->nqb_all;
+    p->qdelta = kf % 2;
+    p->npairs = p->G;
+    p->units = B * Hkv * p->npairs;
+    p->nqb = (p->nqb_all + p->qdelta + 1) / 2;
+  }
   // Persistent grid. Item cost = (visited tiles + fixed per-item overhead,
   // about the pipeline fill/drain and epilogue) x Q tiles of the item; it is
   // used to find the heavy q-blocks, how finely to cut them, and how many
@@ -1336,9 +1382,25 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
   const int grid = static_cast<int>(std::min<long long>(std::min(max_ctas, kMaxCtas), n_items));
   std::vector<long long> qcost(p->nqb);
   long long total = 0;
+  // (per-head bands: the heavy items and the split are chosen from the costs
+  // at the maximal band, as the workspace query sees them; the rounds the
+  // CTAs holding an extra heavy item sit out are counted from the heads' own
+  // mean costs, in mcost)
+  // (with q-block pairs an item holds 1 or 2 Q tiles, one item per head and
+  // pair: the costs below are then per item, both Q tiles included)
+  std::vector<long long> mcost(p->nqb);
   for (int qb = 0; qb < p->nqb; ++qb) {
-    qcost[qb] = block_tiles(p->pat, p->qb0 + qb, BM, BN).count() + kItemOverheadTiles;
+    const int x = p->qb0 + qb, qa = 2 * x - p->qdelta;
+    const int nq = p->qpair ? (qa >= 0 ? 1 : 0) + (qa + 1 < p->nqb_all ? 1 : 0) : 1;
+    qcost[qb] = (sched_tiles(*p, p->pat, x).count() + kItemOverheadTiles) * nq;
     total += qcost[qb] * static_cast<long long>(B) * Hq;
+    mcost[qb] = qcost[qb];
+    if (hS && hW) {
+      long long sum = 0;
+      for (int h = 0; h < Hq; ++h)
+        sum += sched_tiles(*p, make_pattern(N, 0, hS[h], hW[h], pat.L), x).count();
+      mcost[qb] = ((sum + Hq / 2) / Hq + kItemOverheadTiles) * nq;
+    }
   }
   const double target = static_cast<double>(total) / grid;
   // heavy q-blocks: from the top, while an item of the block costs more than a
@@ -1346,7 +1408,7 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
   // CTA that drew such an item in the strided rounds would carry its excess;
   // dealt first, its holders join the rounds late instead); at most 8 big
   // items per CTA
-  const long long item_q = p->G >= 2 ? 2 : 1;
+  const long long item_q = p->qpair ? 1 : (p->G >= 2 ? 2 : 1);
   std::vector<long long> sorted_cost(qcost);
   std::nth_element(sorted_cost.begin(), sorted_cost.begin() + p->nqb / 2, sorted_cost.end());
   const long long median = sorted_cost[p->nqb / 2];
@@ -1367,11 +1429,11 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
   if (split && !sparse && n_hqb > 0) {
     const double heavy = static_cast<double>(qcost[p->nqb - 1] * item_q);
     ns = static_cast<int>(std::ceil(heavy / (kSplitShare * target)));
-    ns = std::min(ns, std::max(1, block_tiles(p->pat, p->qb0 + p->nqb - 1, BM, BN).count() /
+    ns = std::min(ns, std::max(1, sched_tiles(*p, p->pat, p->qb0 + p->nqb - 1).count() /
                                       kMinPieceTiles));
     ns = std::min(ns, kMaxSplit);
     while (n_sqb < n_hqb && qcost[p->nqb - 1 - n_sqb] * item_q > kSplitShare * target &&
-           block_tiles(p->pat, p->qb0 + p->nqb - 1 - n_sqb, BM, BN).count() >= ns * kMinPieceTiles)
+           sched_tiles(*p, p->pat, p->qb0 + p->nqb - 1 - n_sqb).count() >= ns * kMinPieceTiles)
       ++n_sqb;
     ns = std::min(ns, std::max(1, static_cast<int>(
                               (8LL * grid - (n_hqb - n_sqb) * static_cast<long long>(p->units)) /
@@ -1385,12 +1447,18 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
   // per stride of grid items a digit of radix n advances by d (plus carries)
   // and the q-block slot by d_qi; the first rotation r that makes d + d_qi * r
   // coprime with n lets that digit run through all its values
+  // (a stride's q-block slot advance is d_qi, or d_qi + 1 when the lower
+  // digits carry; a rotation that makes either advance coprime with n moves
+  // the digit through all its values over the CTA's items)
   auto coprime_rotation = [](int d, int d_qi, int n) {
-    for (int r = 0; r < n; ++r) {
-      int a = (d + d_qi * r) % n, b = n;
+    auto coprime = [](int a, int b) {
       while (b) { const int t = a % b; a = b; b = t; }
-      if (a == 1) return r;
-    }
+      return a == 1;
+    };
+    for (int r = 0; r < n; ++r)
+      if (coprime((d + d_qi * r) % n, n)) return r;
+    for (int r = 0; r < n; ++r)
+      if (coprime((d + (d_qi + 1) * r) % n, n)) return r;
     return 0;
   };
   if (p->pat.causal && !sparse && !mix_pairs && p->G % 2 == 0 && n_hqb == 0 && grid >= p->npairs) {
@@ -1410,10 +1478,10 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
     // others spend on an equal cost of normal items
     double big_cost = 0, norm_cost = 0;
     for (int q = 0; q < n_hqb; ++q)
-      big_cost += qcost[p->nqb - 1 - q] +
+      big_cost += mcost[p->nqb - 1 - q] +
                   (q < n_sqb ? ns * kSplitOverheadTiles + (ns - 1) * kItemOverheadTiles : 0);
     big_cost = big_cost * B * Hq / p->n_big;
-    for (int qb = 0; qb < p->nqb - n_hqb; ++qb) norm_cost += qcost[qb];
+    for (int qb = 0; qb < p->nqb - n_hqb; ++qb) norm_cost += mcost[qb];
     norm_cost = norm_cost * B * Hq / n_norm;
     p->n_a = p->n_big % grid;
     const double rounds = big_cost / norm_cost;
@@ -1463,7 +1531,7 @@ int launch_attention_d(const LaunchArgs& a, DeviceInfo* di) {
   const bool sparse = a.bs_off != nullptr;
   // per-head bands: pairs differ in cost, so every CTA cycles through the pairs
   const int grid = build_schedule(a.B, a.Hq, a.Hkv, a.N, a.pat, di->sms, a.ws != nullptr, &p,
-                                  sparse, a.hS != nullptr, a.qb_lo, a.qb_hi - a.qb_lo);
+                                  sparse, a.hS != nullptr, a.qb_lo, a.qb_hi - a.qb_lo, a.hS, a.hW);
   p.sl2 = a.scale * 1.4426950408889634f;
   p.inject_cta = a.inject_cta;
   if (a.hS) {  // per-head bands; a.pat already holds the maxima
@@ -1606,14 +1674,20 @@ int workspace_bytes(int B, int Hq, int Hkv, int N, int D, const Pattern& pat, in
   AttnParams p;
   build_schedule(B, Hq, Hkv, N, pat, num_ctas, true, &p);
   *bytes = ws_layout(p, D).total;
+  if (!pat.causal) {  // per-head band launches of the same (maximal) band pair q-blocks
+    AttnParams ph;
+    build_schedule(B, Hq, Hkv, N, pat, num_ctas, true, &ph, false, true);
+    *bytes = std::max(*bytes, ws_layout(ph, D).total);
+  }
   return TM_OK;
 }
 
 int debug_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ctas, int split,
-                   int qb_lo, int qb_hi, int* out, long long cap, long long* count) {
+                   int qb_lo, int qb_hi, int* out, long long cap, long long* count, const int* hS,
+                   const int* hW) {
   AttnParams p;
   const int grid = build_schedule(B, Hq, Hkv, N, pat, max_ctas, (split & 1) != 0, &p, false,
-                                  (split & 2) != 0, qb_lo, qb_hi - qb_lo);
+                                  (split & 2) != 0, qb_lo, qb_hi - qb_lo, hS, hW);
   long long n = 0;
   for (int c = 0; c < grid; ++c) {
     const int n_work = work_count(p, c, grid);
@@ -1621,9 +1695,12 @@ int debug_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
       const Item it = work_item_at(p, c, grid, k);  // what the producer publishes
       const int item = work_item(p, c, grid, k);
       if (n >= cap) continue;
-      const int T = block_tiles(p.pat, it.qb, BM, BN).count();
+      const int T = item_tiles(p, it).count();
       int* r = out + 7 * n;
-      r[0] = c; r[1] = item; r[2] = it.qb; r[3] = it.b * Hq + it.h0; r[4] = 1 + it.v1;
+      // Q tiles: heads h0, h0 + 1 of q-block qb, or (q-block pairs, bit 8 set)
+      // q-blocks qb, qb + 1 of head h0
+      r[0] = c; r[1] = item; r[2] = it.qb; r[3] = it.b * Hq + it.h0;
+      r[4] = 1 + it.v1 + (p.qpair ? 256 : 0);
       r[5] = it.t0; r[6] = std::min(T, it.t1);
     }
   }

@@ -56,7 +56,8 @@ long long kernel_launches();
 int launch_discovery(const DiscArgs& a);
 long long discovery_workspace_bytes(int B, int Hq, int Hkv, int N, int D, int P);
 int debug_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ctas, int split,
-                   int qb_lo, int qb_hi, int* out, long long cap, long long* count);
+                   int qb_lo, int qb_hi, int* out, long long cap, long long* count,
+                   const int* hS = nullptr, const int* hW = nullptr);
 // Workspace bytes the split schedule needs on num_ctas CTAs (<= 0: the
 // current device's SM count); 0 if no item is split.
 int workspace_bytes(int B, int Hq, int Hkv, int N, int D, const Pattern& pat, int num_ctas,

@@ -51,9 +51,9 @@ struct BlockTiles {
   TM_HD int kb(int t) const { return t < n_a ? t : b_lo + (t - n_a); }
 };
 
-TM_HD BlockTiles block_tiles(const Pattern& p, int qb, int BM, int BN) {
-  const int r0 = qb * BM;
-  const int r1 = imin(p.N, r0 + BM) - 1;
+// Kept k-blocks of the query rows [r0, r1] (r1 < N): the union of their kept
+// keys, which is the closed form at the block's first and last rows.
+TM_HD BlockTiles block_tiles_rows(const Pattern& p, int r0, int r1, int BN) {
   const int last = r1 / BN;
   BlockTiles t;
   if (p.causal || r1 >= p.N - p.L) {
@@ -69,6 +69,10 @@ TM_HD BlockTiles block_tiles(const Pattern& p, int qb, int BM, int BN) {
     t.n_a = n_sink; t.b_lo = b_lo; t.n_b = last - b_lo + 1;
   }
   return t;
+}
+
+TM_HD BlockTiles block_tiles(const Pattern& p, int qb, int BM, int BN) {
+  return block_tiles_rows(p, qb * BM, imin(p.N, qb * BM + BM) - 1, BN);
 }
 
 // 1 iff every pair of the tile's existing rows [r0, r1] and columns [c0, c1] is

@@ -194,25 +194,55 @@ def test_items_of_one_kv_head_and_q_block_are_adjacent(B, Hq, Hkv, N, causal, W,
         assert max(items) - min(items) == npairs - 1, (key, sorted(items))
 
 
+def union_tiles(N, causal, S, W, L, r0, r1):
+    """Key blocks holding a kept key of any row in [r0, r1] (the union list of a
+    q-block pair), from the pattern's per-row intervals: every causal key for
+    causal rows and the last L rows, else the sinks [0, S) and the window
+    [i - W + 1, i], whose ends grow with i."""
+    if causal or r1 >= N - L:
+        return r1 // 128 + 1
+    blocks = set(range((min(S, r1 + 1) + 127) // 128))
+    blocks.update(range(max(0, r0 - W + 1) // 128, r1 // 128 + 1))
+    return len(blocks)
+
+
 @pytest.mark.parametrize("B,Hq,Hkv,N,causal,S,W,L", CASES[:12] + SPLIT_CASES[:4])
 def test_pair_and_kv_rotation_keep_exact_coverage(B, Hq, Hkv, N, causal, S, W, L):
-    # per-head band launches rotate the pair and kv-head digits per q-block; the
-    # host export cross-checks the device cursor against the direct decode, and
-    # every (q-block, head) must still be covered exactly once, with the items of
-    # one kv head and q-block adjacent
+    # per-head band launches rotate the pair and kv-head digits per q-block and
+    # (for non-causal patterns) pair two consecutive q-blocks of one head in an
+    # item; every (q-block, head) must still be covered exactly once, and the
+    # pieces of an item must cover its tile list (the union of its Q tiles')
+    nqb = (N + 127) // 128
     for split in (False, True):
         rec = tm.tm_debug_schedule(B, Hq, Hkv, N, causal, S, W, L, 148, split=split, mix_pairs=True)
-        tiles = tm.tm_tile_list(N, causal, S, W, L)
-        per_qb = np.bincount(tiles[:, 0], minlength=(N + 127) // 128)
-        seen = {}
+        ranges = {}
         for c, item, qb, h0, nv, t0, t1 in rec:
-            for h in range(h0, h0 + nv):
-                seen.setdefault((qb, h), []).append((t0, t1))
-        assert len(seen) == ((N + 127) // 128) * B * Hq
-        for (qb, h), ranges in seen.items():
-            ranges.sort()
-            assert ranges[0][0] == 0 and ranges[-1][1] == per_qb[qb]
-            assert all(a1 == b0 for (_, a1), (b0, _) in zip(ranges, ranges[1:]))
+            qpair, nq = nv >> 8, nv & 255
+            assert qpair == (0 if causal else 1)
+            tiles = [(qb + k, h0) for k in range(nq)] if qpair else [(qb, h0 + k) for k in range(nq)]
+            ranges.setdefault(tuple(tiles), []).append((t0, t1))   # the pieces of one item
+        seen = [t for tiles in ranges for t in tiles]
+        assert len(seen) == len(set(seen)) == nqb * B * Hq
+        for tiles, rg in ranges.items():
+            rg.sort()
+            qbs = sorted({t[0] for t in tiles})
+            n_union = union_tiles(N, causal, S, W, L, qbs[0] * 128, min(N, (qbs[-1] + 1) * 128) - 1)
+            assert rg[0][0] == 0 and rg[-1][1] == n_union, (tiles, rg, n_union)
+            assert all(a1 == b0 for (_, a1), (b0, _) in zip(rg, rg[1:]))
+
+
+@pytest.mark.parametrize("N,S,W,L", [(131072, 64, 4096, 256), (131072, 64, 4096, 128),
+                                     (32768, 64, 4096, 128), (1000, 0, 300, 100)])
+def test_qblock_pairs_waste_at_most_one_tile_per_q_tile(N, S, W, L):
+    # a q-block pair's union list holds at most one tile more than each of its
+    # two q-blocks' own lists (the neighbour's band edge or diagonal); the
+    # q-block whose list is full causal (last-L rows) starts a pair
+    per_qb = np.bincount(tm.tm_tile_list(N, False, S, W, L)[:, 0], minlength=(N + 127) // 128)
+    rec = tm.tm_debug_schedule(1, 8, 2, N, False, S, W, L, 148, mix_pairs=True)
+    for c, item, qb, h0, nv, t0, t1 in rec:
+        nq = nv & 255
+        for k in range(nq):
+            assert t1 - per_qb[qb + k] <= 1, (qb, k, t1, per_qb[qb + k])
 
 
 @pytest.mark.parametrize("W", [512, 2048, 4096, 8192, 16384, 32768])
@@ -273,3 +303,20 @@ def test_window_arguments_rejected():
     assert L.tm_debug_schedule_window(1, 4, 2, 1000, 1, 0, 1, 0, 148, 0, 3, -1, None, 0,
                                       ctypes.byref(cnt)) == tm.TM_OK
     assert cnt.value == 5 * 2 * 1
+
+
+@pytest.mark.parametrize("N,L", [(131072, 256), (65536, 128), (32768, 128)])
+def test_per_head_band_schedule_is_balanced(N, L):
+    # the seeded per-head bands of the bench (windows 512..4096, sinks {0, 64}) on
+    # the Llama-3-8B head layout: items are q-block pairs of one head; the heads
+    # rotate across the CTAs, and the CTAs that hold a heavy (last-L) item sit
+    # out rounds worth the heads' mean cost
+    Hq, Hkv = 32, 8
+    hS, hW = I.head_bands(Hq, 0)
+    rec = tm.tm_debug_schedule_heads(1, Hq, Hkv, N, hS, hW, L, 148)
+    cost = np.zeros(148)
+    for c, item, qb, h0, nv, t0, t1 in rec:
+        nq = nv & 255
+        u = union_tiles(N, False, int(hS[h0]), int(hW[h0]), L, qb * 128, min(N, (qb + nq) * 128) - 1)
+        cost[c] += (min(u, t1) - t0 + 3) * nq
+    assert cost.max() / cost.mean() <= 1.08, cost.max() / cost.mean()
