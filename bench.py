@@ -40,7 +40,7 @@ BM = BN = 128
 # triangle launch of the default workload (llama3-8b-128k, W=2048) from a
 # one-launch ncu capture, keyed by the hash of the build inputs it was taken
 # on; reported only while the sources still match (else null).
-TRAFFIC: dict = {"d5a80b5dc5102fc4": 2171954176 + 1042875136}
+TRAFFIC: dict = {"e1d9740743a435db": 2260508160 + 1045925888}
 
 
 def _code_only(text: str) -> str:
