@@ -358,7 +358,8 @@ TM_API int tm_debug_mma_probe(const void* q, const void* k, const void* v, float
  * item is a piece). An item covers one q-block of one or two q heads that
  * share a kv head; with q-block pairs (Q tiles has bit 8 set, 256 + 1 or 256 +
  * 2), one or two consecutive q-blocks of one head, whose tile list is the
- * union of theirs. out: HOST buffer of 7*cap ints (NULL when cap = 0); *count
+ * union of theirs. Causal schedules of an odd group size (Hq / Hkv odd, above
+ * 1) over all q-blocks use q-block pairs too. out: HOST buffer of 7*cap ints (NULL when cap = 0); *count
  * receives the total. Host only.
  */
 TM_API int tm_debug_schedule(int B, int Hq, int Hkv, int N, int causal, int S, int W, int L,

@@ -219,13 +219,18 @@ struct AttnParams {
   // item visits the union of its two heads' tile lists, which is the closed
   // form at (max S, max W) since both kept sets are [0, S) U [i - W + 1, i].
   int ph;
-  // Q-block pairs (qpair != 0: per-head band launches): the two Q tiles of an
-  // item are consecutive q-blocks qb, qb + 1 of one q head instead of two
-  // heads of a group, so the union of their tile lists wastes about one tile
-  // per Q tile (heads of one group can have very different bands). The
-  // schedule's q-block x is then the pair of q-blocks 2x - qdelta, 2x + 1 -
-  // qdelta (qdelta puts the first full-causal q-block of the last-L rows at
-  // the start of a pair); a pair cut by the sequence's ends holds one Q tile.
+  // Q-block pairs (qpair != 0): the two Q tiles of an item are consecutive
+  // q-blocks qb, qb + 1 of one q head instead of two heads of a group. Per-head
+  // band launches use them because heads of one group can have very different
+  // bands, while the union of two neighbouring q-blocks' lists wastes about one
+  // tile per Q tile. Causal launches with an odd group size use them because a
+  // head pair would leave one head of every group alone in an item, with one
+  // softmax warpgroup idle; for causal rows the union is the later q-block's
+  // list, one tile more than the earlier one's. The schedule's q-block x is
+  // then the pair of q-blocks 2x - qdelta, 2x + 1 - qdelta (qdelta puts the
+  // first full-causal q-block of the last-L rows at the start of a pair, and
+  // for causal launches leaves q-block 0 alone when the count is odd); a pair
+  // cut by the sequence's ends holds one Q tile.
   int qpair, qdelta;
   int hS[kMaxBandHeads], hW[kMaxBandHeads];
   unsigned char hperm[kMaxBandHeads];
@@ -283,6 +288,22 @@ __host__ __device__ __forceinline__ void pair_heads(const AttnParams& p, int g, 
   it.h1 = it.v1 ? (p.ph ? p.hperm[hp + 1] : hp + 1) : it.h0;
 }
 
+// The Q tiles of unit digit pr of kv head g at schedule q-block x: head pair pr
+// of q-block x, or with q-block pairs the q-blocks 2x - qdelta, 2x + 1 - qdelta
+// of head pr.
+__host__ __device__ __forceinline__ void unit_tiles(const AttnParams& p, int x, int g, int pr,
+                                                    Item& it) {
+  if (p.qpair) {
+    const int qa = 2 * x - p.qdelta;
+    it.qb = imax(qa, 0);
+    it.v1 = (qa >= 0 && qa + 1 < p.nqb_all) ? 1 : 0;
+    it.h0 = it.h1 = g * p.G + pr;
+  } else {
+    it.qb = x;
+    pair_heads(p, g, pr, it);
+  }
+}
+
 // Pattern of one q head, and of an item (the union of its heads' patterns).
 __host__ __device__ __forceinline__ Pattern head_pattern(const AttnParams& p, int h) {
   Pattern q = p.pat;
@@ -323,7 +344,7 @@ __host__ __device__ __forceinline__ Item decode_item(const AttnParams& p, int it
   Item it;
   const int qi = item / p.units;
   const int u = item - qi * p.units;
-  it.qb = p.qb0 + p.nqb - 1 - qi;  // longest q-blocks first
+  const int x = p.qb0 + p.nqb - 1 - qi;  // longest q-blocks first
   // unit digits, fastest first: pair, kv head, batch. The pairs of one kv head
   // and q-block are consecutive items, which the strided rounds hand to
   // neighbouring CTAs: they walk the same tile list in lockstep, so each K/V
@@ -333,14 +354,7 @@ __host__ __device__ __forceinline__ Item decode_item(const AttnParams& p, int it
   const int gb = u / p.npairs;
   it.g = (gb % p.Hkv + static_cast<int>(static_cast<long long>(qi) * p.kv_rot % p.Hkv)) % p.Hkv;
   it.b = gb / p.Hkv;
-  if (p.qpair) {  // q-block pair (qa, qa + 1) of head pr of kv group g
-    const int qa = 2 * it.qb - p.qdelta;
-    it.qb = imax(qa, 0);
-    it.v1 = (qa >= 0 && qa + 1 < p.nqb_all) ? 1 : 0;
-    it.h0 = it.h1 = it.g * p.G + pr;
-  } else {
-    pair_heads(p, it.g, pr, it);
-  }
+  unit_tiles(p, x, it.g, pr, it);
   it.t0 = 0;
   it.t1 = kAllTiles;
   it.split = -1;
@@ -417,10 +431,9 @@ __host__ __device__ __forceinline__ Item normal_item(const AttnParams& p, long l
   const int r2 = rem - gb * per_gb;
   const int qi = p.n_hqb + k * p.qchunk + r2 / p.npairs;
   Item it;
-  it.qb = p.qb0 + p.nqb - 1 - qi;
   it.g = gb % p.Hkv;
   it.b = gb / p.Hkv;
-  pair_heads(p, it.g, r2 % p.npairs, it);
+  unit_tiles(p, p.qb0 + p.nqb - 1 - qi, it.g, r2 % p.npairs, it);
   it.t0 = 0;
   it.t1 = kAllTiles;
   it.split = -1;
@@ -1368,11 +1381,13 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
   p->qchunk = 1;
   p->qpair = 0;
   p->qdelta = 0;
-  if (mix_pairs && !sparse && !pat.causal && qb0 == 0 && (nqb_w < 0 || nqb_w == p->nqb_all)) {
-    // per-head band launches: items are q-block pairs of one head; the first
-    // q-block whose list is full causal (it holds last-L rows) starts a pair
+  const bool whole = qb0 == 0 && (nqb_w < 0 || nqb_w == p->nqb_all);
+  if (!sparse && whole && ((mix_pairs && !pat.causal) || (pat.causal && !mix_pairs && p->G % 2 == 1 && p->G > 1))) {
+    // per-head band launches, and causal launches of odd groups: items are
+    // q-block pairs of one head; the first q-block whose list is full causal
+    // (it holds last-L rows; q-block 0 in a causal launch) starts a pair
     p->qpair = 1;
-    const int kf = p->pat.L > 0 ? (N - p->pat.L) / BM : p->nqb_all;
+    const int kf = (!pat.causal && p->pat.L > 0) ? (N - p->pat.L) / BM : p->nqb_all;
     p->qdelta = kf % 2;
     p->npairs = p->G;
     p->units = B * Hkv * p->npairs;
@@ -1383,7 +1398,7 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
   // used to find the heavy q-blocks, how finely to cut them, and how many
   // rounds the CTAs holding an extra heavy piece sit out.
   const long long n_items = static_cast<long long>(p->nqb) * p->units;
-  const int grid = static_cast<int>(std::min<long long>(std::min(max_ctas, kMaxCtas), n_items));
+  int grid = static_cast<int>(std::min<long long>(std::min(max_ctas, kMaxCtas), n_items));
   std::vector<long long> qcost(p->nqb);
   long long total = 0;
   // (per-head bands: the heavy items and the split are chosen from the costs
@@ -1465,9 +1480,15 @@ int build_schedule(int B, int Hq, int Hkv, int N, const Pattern& pat, int max_ct
       if (coprime((d + (d_qi + 1) * r) % n, n)) return r;
     return 0;
   };
-  if (p->pat.causal && !sparse && !mix_pairs && p->G % 2 == 0 && n_hqb == 0 && grid >= p->npairs) {
+  // (chunked order: items of one turn must cost alike, so the group is even
+  // or its items are q-block pairs)
+  if (p->pat.causal && !sparse && !mix_pairs && (p->G % 2 == 0 || p->qpair) && n_hqb == 0 &&
+      grid >= p->npairs) {
     p->gchunk = 1;
     p->qchunk = grid / p->npairs;
+    // one turn per round exactly: with 7 heads a group's turn is 147 items, and
+    // a 148th CTA would shift the turn boundary by one item every round
+    grid = p->qchunk * p->npairs;
   }
   const int d_qi = grid / p->units;
   if (!p->gchunk && (p->G % 2 == 1 || mix_pairs) && p->npairs > 1)

@@ -64,6 +64,7 @@ SMALL = [  # B, Hq, Hkv, N, D, S, W, L, causal
     (2, 3, 1, 3001, 128, 1, 64, 1000, False),   # odd group, ragged N, two batches
     (1, 2, 1, 8192, 64, 16, 256, 300, False),   # D = 64 records
     (1, 2, 1, 6000, 128, 0, 1, 0, True),        # causal, few heads
+    (2, 3, 1, 3129, 128, 0, 1, 0, True),        # causal odd group: q-block pairs, q-block 0 alone
 ]
 
 

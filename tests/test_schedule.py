@@ -24,21 +24,41 @@ CASES += [(1, 2, 1, 1, False, 0, 1, 0), (3, 4, 1, 383, False, 1, 1, 1), (1, 14, 
           (2, 6, 2, 129, True, 0, 1, 0), (8, 32, 8, 4096, False, 64, 1024, 128)]
 
 
+def rec_tiles(qb, h0, nv):
+    """The (q-block, q head) Q tiles of a schedule record: a pair of heads of one
+    q-block, or (bit 8 of the count) consecutive q-blocks of one head."""
+    qpair, nq = nv >> 8, nv & 255
+    return [(qb + k, h0) for k in range(nq)] if qpair else [(qb, h0 + k) for k in range(nq)]
+
+
+def qblock_pairs(Hq, Hkv, causal):
+    """Causal launches of odd groups pair two q-blocks of one head per item."""
+    G = Hq // Hkv
+    return causal and G % 2 == 1 and G > 1
+
+
+def n_items_whole(B, Hq, Hkv, N, causal):
+    G, nqb = Hq // Hkv, (N + 127) // 128
+    if qblock_pairs(Hq, Hkv, causal):
+        return (nqb + 1) // 2 * B * Hq
+    return nqb * B * Hkv * ((G + 1) // 2)
+
+
 @pytest.mark.parametrize("B,Hq,Hkv,N,causal,S,W,L", CASES)
 def test_every_item_exactly_once(B, Hq, Hkv, N, causal, S, W, L):
     rec = tm.tm_debug_schedule(B, Hq, Hkv, N, causal, S, W, L, 148)
-    G = Hq // Hkv
     nqb = (N + 127) // 128
-    n_items = nqb * B * Hkv * ((G + 1) // 2)
+    n_items = n_items_whole(B, Hq, Hkv, N, causal)
     assert len(rec) == n_items
     assert sorted(rec[:, 1].tolist()) == list(range(n_items))
+    assert ((rec[:, 4] >> 8) == int(qblock_pairs(Hq, Hkv, causal))).all()
     # every (batch, q head, q-block) tile appears once
     tiles = set()
     for c, item, qb, h0, nv, t0, t1 in rec:
         assert t0 == 0
-        for h in range(h0, h0 + nv):
-            assert (qb, h) not in tiles
-            tiles.add((qb, h))
+        for t in rec_tiles(qb, h0, nv):
+            assert t not in tiles
+            tiles.add(t)
     assert len(tiles) == nqb * B * Hq
     # the grid never exceeds the SM count or the item count
     assert rec[:, 0].max() < min(148, n_items)
@@ -96,27 +116,49 @@ def test_concurrent_items_share_kv_tiles(N, causal, W, L):
 
 
 @pytest.mark.parametrize("N,Hq,Hkv", [(131072, 32, 8), (65536, 32, 8), (32768, 32, 8),
-                                      (131072, 4, 1), (65536, 8, 2)])
+                                      (131072, 4, 1), (65536, 8, 2), (131072, 28, 4),
+                                      (65536, 28, 4), (131072, 7, 1)])
 def test_causal_chunked_group_order_is_balanced(N, Hq, Hkv):
     rec = tm.tm_debug_schedule(1, Hq, Hkv, N, True, 0, 1, 0, 148)
     cost = np.zeros(148)
     for c, item, qb, h0, nv, t0, t1 in rec:
-        cost[c] += (qb + 1 + 3) * nv
+        last = max(q for q, _ in rec_tiles(qb, h0, nv))
+        cost[c] += (last + 1 + 3) * (nv & 255)
     assert cost.max() / cost.mean() <= 1.01, cost.max() / cost.mean()
+
+
+@pytest.mark.parametrize("N,Hq,Hkv", [(131072, 28, 4), (65536, 28, 4), (131072, 7, 1)])
+def test_odd_group_causal_rounds_read_one_kv_head(N, Hq, Hkv):
+    # Groups of 7 heads: items pair two q-blocks of one head, 7 per kv head and
+    # slot; a turn of 21 slots is 147 items, and the grid is 147 CTAs, so every
+    # round of the full chunks reads one kv head's K/V (64 MB at 128K, in L2)
+    G = Hq // Hkv
+    rec = tm.tm_debug_schedule(1, Hq, Hkv, N, True, 0, 1, 0, 148)
+    grid = rec[:, 0].max() + 1
+    assert grid == 148 // G * G
+    order = np.argsort(rec[:, 1])
+    kvh, qbs = rec[order, 3] // G, rec[order, 2]
+    nslots = (N // 128 + 1) // 2
+    full = nslots // (grid // G) * (grid // G) * G * Hkv   # items of the full chunks
+    for r0 in range(0, full, grid):
+        assert len(set(kvh[r0:r0 + grid].tolist())) == 1, r0
+        assert qbs[r0:r0 + grid].max() - qbs[r0:r0 + grid].min() < 2 * (grid // G) + 1, r0
 
 
 SPLIT_CASES = [(1, 4, 1, 131072, False, 64, 2048, 256), (1, 4, 1, 131072, False, 64, 512, 256),
                (1, 8, 2, 65536, False, 64, 1024, 128), (1, 32, 8, 131072, False, 64, 512, 256),
                (1, 4, 1, 131072, True, 0, 1, 0), (1, 2, 1, 32768, True, 0, 1, 0),
                (1, 4, 4, 512, False, 16, 64, 64), (2, 6, 2, 1000, False, 3, 100, 300),
-               (1, 28, 4, 131072, False, 64, 1024, 128), (1, 7, 1, 65536, False, 64, 1024, 200)]
+               (1, 28, 4, 131072, False, 64, 1024, 128), (1, 7, 1, 65536, False, 64, 1024, 200),
+               (2, 3, 1, 3129, True, 0, 1, 0), (1, 5, 1, 20000, True, 0, 1, 0)]
 
 
 def cta_costs(rec, per_qb, n_ctas=148, overhead=3, split_overhead=1):
     cost = np.zeros(n_ctas)
     for c, item, qb, h0, nv, t0, t1 in rec:
-        piece = (t1 - t0) + overhead + (split_overhead if t1 - t0 < per_qb[qb] else 0)
-        cost[c] += piece * nv
+        n_union = max(per_qb[q] for q, _ in rec_tiles(qb, h0, nv))
+        piece = (t1 - t0) + overhead + (split_overhead if t1 - t0 < n_union else 0)
+        cost[c] += piece * (nv & 255)
     return cost
 
 
@@ -125,22 +167,25 @@ def test_split_pieces_cover_each_item_once(B, Hq, Hkv, N, causal, S, W, L):
     rec = tm.tm_debug_schedule(B, Hq, Hkv, N, causal, S, W, L, 148, split=True)
     tiles = tm.tm_tile_list(N, causal, S, W, L)
     per_qb = np.bincount(tiles[:, 0], minlength=(N + 127) // 128)
-    seen = {}
+    seen, end = {}, {}
     for c, item, qb, h0, nv, t0, t1 in rec:
-        assert 0 <= t0 < t1 <= per_qb[qb]
-        for h in range(h0, h0 + nv):
-            seen.setdefault((qb, h), []).append((t0, t1))
+        tiles = rec_tiles(qb, h0, nv)
+        n_union = max(per_qb[q] for q, _ in tiles)   # the item's list covers its Q tiles' lists
+        assert 0 <= t0 < t1 <= n_union
+        for t in tiles:
+            seen.setdefault(t, []).append((t0, t1))
+            end[t] = n_union
     nqb = (N + 127) // 128
     assert len(seen) == nqb * B * Hq
     for (qb, h), ranges in seen.items():
         ranges.sort()
-        assert ranges[0][0] == 0 and ranges[-1][1] == per_qb[qb], (qb, h, ranges)
+        assert ranges[0][0] == 0 and ranges[-1][1] == end[(qb, h)], (qb, h, ranges)
         for (a0, a1), (b0, b1) in zip(ranges, ranges[1:]):
             assert a1 == b0, (qb, h, ranges)   # contiguous, no overlap
     # the item ids are a permutation
     assert sorted(rec[:, 1].tolist()) == list(range(len(rec)))
     # pieces of one heavy item run on different CTAs, all before normal work
-    pieces = rec[(rec[:, 6] - rec[:, 5]) < per_qb[rec[:, 2]]]
+    pieces = rec[(rec[:, 6] - rec[:, 5]) < per_qb[np.minimum(rec[:, 2] + (rec[:, 4] >> 8), nqb - 1)]]
     for key in {(int(q), int(h)) for _, _, q, h, _, _, _ in pieces}:
         ctas = pieces[(pieces[:, 2] == key[0]) & (pieces[:, 3] == key[1])][:, 0]
         assert len(set(ctas.tolist())) == len(ctas)
@@ -277,6 +322,7 @@ def test_row_chunk_windows_cover_each_item_once(B, Hq, Hkv, N, causal, S, W, L, 
     for r0 in range(0, N, chunk):
         lo, hi = r0 // 128, (min(N, r0 + chunk) + 127) // 128
         rec = tm.tm_debug_schedule(B, Hq, Hkv, N, causal, S, W, L, 148, qb_lo=lo, qb_hi=hi)
+        # (a window of the rows keeps head pairs: its q-blocks need not pair up)
         assert len(rec) == (hi - lo) * B * Hkv * ((Hq // Hkv + 1) // 2)
         assert rec[:, 2].min() >= lo and rec[:, 2].max() < hi
         # the longest q-blocks of the chunk come first in each CTA (for causal
@@ -286,10 +332,10 @@ def test_row_chunk_windows_cover_each_item_once(B, Hq, Hkv, N, causal, S, W, L, 
             if causal:
                 assert mine[0, 2] == mine[:, 2].max()
         for c, item, qb, h0, nv, t0, t1 in rec:
-            assert t0 == 0
-            for h in range(h0, h0 + nv):
-                assert (qb, h) not in seen
-                seen[(qb, h)] = 1
+            assert t0 == 0 and nv >> 8 == 0
+            for t in rec_tiles(qb, h0, nv):
+                assert t not in seen
+                seen[t] = 1
     assert len(seen) == nqb * B * Hq
 
 
