@@ -117,6 +117,7 @@ EDGE = [  # B, Hq, Hkv, N, D, S, W, L
     (1, 14, 2, 777, 128, 5, 200, 100),
     (3, 4, 1, 383, 64, 1, 1, 1),
     (1, 2, 2, 2049, 128, 64, 300, 129),
+    (2, 6, 2, 1100, 64, 16, 200, 100),  # odd group at D = 64: causal items pair q-blocks
 ]
 
 
