@@ -19,6 +19,12 @@
  * Query head hq reads kv head hq / (Hq / Hkv) (consecutive q heads share a kv
  * head). D must be 64 or 128. RoPE, if any, is applied by the caller.
  *
+ * Numerics: scores and the softmax are fp32, the weights P bf16, and O, l fp32
+ * sums on the tensor cores. The softmax reference (the running max) moves only
+ * when a tile's scores exceed it by more than 48 in the log2 domain, so P stays
+ * below 2^48. O stays finite for |v| up to about 2^62 over 2^17 keys, which is
+ * far outside the range of activations.
+ *
  * Ownership and threading:
  *   - q, k, v, o are DEVICE pointers owned by the caller, 16-byte aligned;
  *     o must not overlap q, k or v (tm_trianglemix_attn_fwd_host takes host

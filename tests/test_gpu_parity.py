@@ -171,6 +171,28 @@ def test_special_unit_values(mid):
     assert np.abs(out - 1.0).max() <= 4e-3
 
 
+def test_special_rising_scores_scale_with_v():
+    """Scores that rise by ~100 log2 units along the keys: the running reference
+    lags the row max by up to the lazy threshold, so weights reach 2^48 before it
+    moves. Attention is linear in v and a power-of-two scale is exact in bf16 and
+    fp32, so v * 2^40 must give the output * 2^40 bit for bit, with no overflow."""
+    B, Hq, Hkv, N, D = 1, 2, 1, 1500, 128
+    q = np.zeros((B, N, Hq, D), np.uint16)
+    q[..., 0] = I.f32_to_bf16_bits(np.float32(16.0))
+    k = np.zeros((B, N, Hkv, D), np.uint16)
+    k[0, :, 0, 0] = I.f32_to_bf16_bits((49.0 * np.arange(N) / N).astype(np.float32))
+    v = rand_bits((B, N, Hkv, D), 41)
+    v40 = I.f32_to_bf16_bits(I.bf16_bits_to_f32(v) * np.float32(2.0 ** 40))
+    scale = 1.0 / math.sqrt(D)
+    for causal, S, W, L in ((True, 0, 1, 0), (False, 3, 900, 200)):
+        out = run(q, k, v, B, Hq, Hkv, N, D, scale, causal, S, W, L)
+        big = run(q, k, v40, B, Hq, Hkv, N, D, scale, causal, S, W, L)
+        assert np.isfinite(big).all()
+        np.testing.assert_array_equal(big, out * np.float32(2.0 ** 40))
+        want = oracle.attention(q, k, v, B, Hq, Hkv, N, D, scale, causal, S, W, L)
+        assert_close(out, want, f"rising scores causal={causal}")
+
+
 def zero_query_expected(vf, pre, N, S, W, L, rows):
     """Closed form for q = 0: the mean of v over each row's kept set (prefix sums).
     vf: v as float64 [B, N, Hkv, D]; pre: its prefix sums along N. Returns [B, rows, Hkv, D]."""
