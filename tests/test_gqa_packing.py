@@ -1,6 +1,6 @@
 """Does packing the q heads of a GQA group into one 128-row tile pay?
 
-The idea (the survey's first "next" item): for the band part of the triangle,
+The idea: for the band part of the triangle,
 put 32 consecutive query rows of each of the G = 4 q heads that share a kv
 head into one M = 128 tile, so that one K/V tile feeds all four heads at once
 and each 32-row slice visits only the key blocks its own rows keep. The saving
