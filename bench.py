@@ -514,7 +514,7 @@ def other_legs(args, wl, W, tm, dq, dk, dv, do, stream, causal_ms, tri_layer):
         },
         "head_bands": {
             "what": "tm_triangle_attn_fwd_heads, seeded per-head windows 512..4096 (log-uniform) "
-                    "and sinks {0, 64}, L shared; heads paired in band order",
+                    "and sinks {0, 64}, L shared; items pair two q-blocks of one head",
             "ms": hb_ms,
             "tflops_own_tiles": head_tiles * 4.0 * BM * BN * wl.D / (hb_ms * 1e-3) / 1e12,
             "own_tiles": int(head_tiles),

@@ -145,9 +145,10 @@ TM_API int tm_trianglemix_attn_fwd_host(const void* q_host, const void* k_host,
  * precision regions computed in bf16 the computed region is one band below
  * the diagonal, here widened by the head's sinks.
  * S_heads, W_heads: HOST arrays of Hq ints (S_h >= 0, W_h >= 1; S_h and W_h
- * larger than N act as N); Hq <= 128. The heads of a kv group are paired in
- * band order and a pair visits the union of its two bands (masked per head),
- * so heads with similar bands cost nothing extra. workspace / workspace_bytes
+ * larger than N act as N); Hq <= 128. Each work item holds two consecutive
+ * q-blocks of one head and visits the union of their tile lists, each Q tile
+ * masked with its own rows, so a Q tile visits at most one tile it does not
+ * need; the heads rotate across the CTAs. workspace / workspace_bytes
  * as for tm_triangle_attn_fwd_ws, sized by tm_attn_workspace_size with
  * S = max S_h and W = max W_h (NULL and 0 split nothing).
  */
