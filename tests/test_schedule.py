@@ -366,3 +366,31 @@ def test_per_head_band_schedule_is_balanced(N, L):
         u = union_tiles(N, False, int(hS[h0]), int(hW[h0]), L, qb * 128, min(N, (qb + nq) * 128) - 1)
         cost[c] += (min(u, t1) - t0 + 3) * nq
     assert cost.max() / cost.mean() <= 1.08, cost.max() / cost.mean()
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_random_causal_odd_groups_cover_each_tile_once(seed):
+    # random shapes of odd group size (q-block pairs of one head), with and without
+    # the split workspace: every (q-block, q head) Q tile is covered exactly once,
+    # and the pieces of an item cover its list (the later q-block's) without gaps
+    rng = np.random.default_rng(seed)
+    G = int(rng.choice([3, 5, 7, 9]))
+    Hkv = int(rng.integers(1, 4))
+    B = int(rng.integers(1, 3))
+    N = int(rng.integers(1, 6000))
+    Hq = G * Hkv
+    nqb = (N + 127) // 128
+    for split in (False, True):
+        rec = tm.tm_debug_schedule(B, Hq, Hkv, N, True, 0, 1, 0, 148, split=split)
+        ranges = {}
+        for c, item, qb, h0, nv, t0, t1 in rec:
+            tiles = tuple(rec_tiles(qb, h0, nv))
+            assert nv >> 8 == (1 if G > 1 else 0) and 1 <= (nv & 255) <= 2
+            ranges.setdefault(tiles, []).append((t0, t1))
+        seen = [t for tiles in ranges for t in tiles]
+        assert len(seen) == len(set(seen)) == nqb * B * Hq, (G, Hkv, B, N, split)
+        for tiles, rg in ranges.items():
+            rg.sort()
+            last = max(q for q, _ in tiles)
+            assert rg[0][0] == 0 and rg[-1][1] == last + 1, (tiles, rg)
+            assert all(a1 == b0 for (_, a1), (b0, _) in zip(rg, rg[1:]))
