@@ -17,9 +17,10 @@
 // (2 x 128 x 208 + 128 x 88 = 64512), so the row of 128 scores stays in
 // registers. The host refuses to launch a build whose register count differs.
 // A work item is (batch, kv head, pair of q heads of that kv head's group,
-// q-block): both Q tiles read the same K/V stream, which is loaded once. Only
-// the kept k-blocks of the q-block are visited (tm_tiles.cuh); elementwise
-// masking runs only on the tiles that need it.
+// q-block), or, in per-head band launches and causal launches of odd group
+// sizes, two consecutive q-blocks of one q head: both Q tiles read the same
+// K/V stream, which is loaded once. Only the kept k-blocks are visited
+// (tm_tiles.cuh); elementwise masking runs only on the tiles that need it.
 //
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).
 // The output leaves through shared memory and TMA stores (one 4 KB slot per
