@@ -53,7 +53,8 @@ def _inputs(B, Hq, Hkv, N, D, seed):
 @pytest.mark.gpu
 @pytest.mark.parametrize("B,Hq,Hkv,N,D,S,W,L", [(1, 4, 1, 32768, 128, 64, 1024, 128),
                                                (1, 2, 1, 4173, 128, 5, 100, 200),
-                                               (1, 2, 1, 8192, 64, 16, 256, 300)])
+                                               (1, 2, 1, 8192, 64, 16, 256, 300),
+                                               (1, 3, 1, 4173, 128, 5, 100, 200)])
 def test_noalloc_matches_workspace_entry_two_calls_in_a_row(B, Hq, Hkv, N, D, S, W, L):
     import torch
     if not torch.cuda.is_available():
